@@ -1,0 +1,375 @@
+#!/usr/bin/env python
+"""Benchmark of the NVFP4 quantized linear on B200 through the libbsp C ABI.
+
+One step = one pass of the hot path over one batch: the NVFP4 activation quantizer
+(bf16 -> E2M1 codes + E4M3 block-16 scales) followed by the block-scaled FP4 GEMM
+with the fused alpha * acc + bias -> bf16 epilogue ("BFL (fp8r / nvfp4)", Kernels
+table).  Default workload: the attention projection of a rectified-flow image
+transformer at 1 MP (4096 tokens, 3072 -> 3072, bias).  Weights are quantized once
+before timing (they are stored pre-quantized); the activation global scale is a
+calibrated constant computed once.
+
+Timing: W untimed warm-up steps, then K steps, each bracketed by CUDA events on the
+launching stream, with the 126 MB L2 flushed (a 256 MiB write) before every step,
+outside the events.  The step's two kernels are each replayed from a CUDA graph.
+Barrier + synchronize around the timed loop; the per-rank total is reduced with MAX.
+With N > 1 (torchrun), every rank runs an independent replica of the same workload
+(the linear shards along tokens with no exchange): value = all ranks' FLOPs / max
+time, "scaling": "weak".
+
+`--impl reference` times the CPU oracle (oracle/) on a bounded sample of rows of
+the same workload, on this host's cores; it is a deliberately slow correctness
+reference, not a competing GPU implementation.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 GEMM TFLOPS & % of B200 FP4 peak; act-quantize GB/s & % of HBM"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    p = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=100)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["bsp", "reference"], default="bsp")
+    p.add_argument("--workload", default="nvfp4_attn_1mp")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=2048,
+                   help="rows of A in the CPU-oracle baseline sample")
+    return p.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def gemm_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("gemm.cu", "bsp_ptx.cuh"):
+        with open(os.path.join(ROOT, "block_scaled_precision_act_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload: str):
+    """DRAM bytes per GEMM launch from the committed ncu summary, if it was taken on
+    the current GEMM source (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    e = d.get(workload)
+    if not e or e.get("source_hash") != gemm_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while the timed loop runs."""
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+               0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+               0x100: "display_clock_setting"}
+
+    def __init__(self, device_index: int):
+        self.samples, self.reasons, self.max_mhz = [], 0, None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._h = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+            except Exception:
+                pass
+            time.sleep(0.001)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._h is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if self._h is None or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"]}
+        names = [n for bit, n in self.REASONS.items() if self.reasons & bit and bit != 0x1]
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(wl, rows: int, A=None, W=None):
+    """Quantize `rows` rows of A and run the fp64 GEMM against the full weight with the
+    oracle, as it stands.  Returns (seconds, flops, threads)."""
+    import numpy as np
+    import oracle
+    import torch
+    A = wl.A() if A is None else A
+    W = wl.W() if W is None else W
+    bias = wl.bias_vec()
+    gw = oracle.nvfp4_global_scale(W)
+    wc, wsf = oracle.nvfp4_quantize(W, gw)          # offline weight prep, untimed
+    ga = oracle.nvfp4_global_scale(A)               # calibrated input scale, untimed
+    rows = min(rows, wl.M)
+    idx = torch.from_numpy(np.linspace(0, wl.M - 1, rows).astype(np.int64))
+    a_rows = A[idx].contiguous()
+    b = None if bias is None else bias.float().numpy().astype(np.float64)
+    t0 = time.perf_counter()
+    ac, asf = oracle.nvfp4_quantize(a_rows, ga)
+    oracle.nvfp4_linear(ac, asf, ga, wc, wsf, gw, b)
+    dt = time.perf_counter() - t0
+    return dt, 2.0 * rows * wl.N * wl.K, oracle.default_threads()
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import synth
+    wl = synth.WORKLOADS[args.workload]
+    A, W = wl.A(), wl.W()
+    # size each step's sample so the whole run stays within a few minutes
+    dt, _, _ = cpu_oracle_sample(wl, 16, A, W)
+    budget_s = 150.0 / max(1, args.steps + args.warmup)
+    rows = int(max(8, min(1024, 16 * budget_s / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        cpu_oracle_sample(wl, rows, A, W)
+    tot, flops, cores = 0.0, 0.0, 1
+    for _ in range(args.steps):
+        dt, fl, cores = cpu_oracle_sample(wl, rows, A, W)
+        tot += dt
+        flops += fl
+    value = flops / tot / 1e12
+    sample = (f"{rows} of {wl.M} rows of A per step (quantize + fp64 GEMM against the "
+              f"full {wl.N}x{wl.K} weight); weight quantization untimed")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K, "bias": wl.bias,
+                   "sample_rows": rows},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------- CUDA path
+def run_bsp(args):
+    import torch
+    import torch.distributed as dist
+    import synth
+    import block_scaled_precision_act_b200 as bsp
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    wl = synth.WORKLOADS[args.workload]
+    if wl.scheme != "nvfp4":
+        raise SystemExit(f"workload {wl.name} is not an NVFP4 linear")
+    M, N, K = wl.M, wl.N, wl.K
+    A_cpu = wl.A()
+    A_host = A_cpu.pin_memory()
+    A = A_cpu.to(dev)
+    W = wl.W().to(dev)
+    bias = wl.bias_vec()
+    bias = None if bias is None else bias.to(dev)
+
+    # untimed preparation: pre-quantized weights and a calibrated activation scale
+    gw = bsp.nvfp4_global_scale(W)
+    wc, wsf = bsp.nvfp4_quantize_act(W, gw, layout=bsp.SF_MMA)
+    ga = bsp.nvfp4_global_scale(A)
+    ac = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+    asf = torch.empty((bsp.nvfp4_sf_bytes(M, K, bsp.SF_MMA),), dtype=torch.uint8, device=dev)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+    flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def quant():
+        bsp.nvfp4_quantize_act(A, ga, codes=ac, scales=asf, layout=bsp.SF_MMA)
+
+    def gemm():
+        bsp.nvfp4_gemm(ac, asf, ga, wc, wsf, gw, bias=bias, out=y)
+
+    quant()
+    gemm()
+    torch.cuda.synchronize(dev)
+    if bsp.bsp_last_device_status() != 0:
+        raise SystemExit("device status not OK after the first step")
+    gq, gg = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(gq, stream=side):
+            quant()
+        with torch.cuda.graph(gg, stream=side):
+            gemm()
+    stream.wait_stream(side)
+    torch.cuda.synchronize(dev)
+
+    n_ev = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        gq.replay()
+        gg.replay()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    sampler = ClockSampler(local)
+    with sampler:
+        for i in range(args.steps):
+            flush.fill_(1)
+            ev[i][0].record(stream)
+            gq.replay()
+            ev[i][1].record(stream)
+            gg.replay()
+            ev[i][2].record(stream)
+        torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    q_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    g_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    s_ms = [e[0].elapsed_time(e[2]) for e in ev]
+    total_ms = sum(s_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if bsp.bsp_last_device_status() != 0:
+        raise SystemExit("device status not OK after the timed steps")
+    if not torch.isfinite(y.float()).all():
+        raise SystemExit("non-finite output")
+
+    # end to end through the public API: pinned host A in, host Y out, every step
+    e2e_steps = max(5, min(args.steps, 50))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    for i in range(e2e_steps + 2):
+        if i == 2:
+            e0.record(stream)
+        A.copy_(A_host, non_blocking=True)
+        quant()
+        gemm()
+        y_host.copy_(y, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    flops = 2.0 * M * N * K
+    ms_per_step = total_ms / args.steps
+    q_mean = statistics.mean(q_ms)
+    g_mean = statistics.mean(g_ms)
+    pk, pk_src = peaks()
+    hbm = pk["hbm_gbs"]
+    fp4_peak = 4.0 * pk["bf16_tflops"]          # nominal fp4 : bf16 dense ratio = 9 : 2.25
+    q_bytes = M * K * 2.5625                    # 2 B read + 0.5 B codes + 1/16 B scales per element
+    gemm_tflops = flops / (g_mean * 1e-3) / 1e12
+    q_gbs = q_bytes / (q_mean * 1e-3) / 1e9
+    traffic = ncu_traffic(wl.name)
+    line = {
+        "metric": METRIC,
+        "value": world * flops / (ms_per_step * 1e-3) / 1e12,
+        "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": wl.name, "M": M, "N": N, "K": K, "bias": wl.bias,
+                   "step": "nvfp4_quantize_act + nvfp4_gemm (fused alpha, bias, bf16)",
+                   "l2": "flushed before every step (256 MiB write, outside the events)",
+                   "parallelism": "replicas" if world > 1 else "single"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
+                     "kernel": "nvfp4_gemm",
+                     "peak_source": f"{pk_src}: 4 x bf16 burst {pk['bf16_tflops']} TFLOP/s "
+                                    "(nominal dense fp4:bf16 = 4)"},
+        "kernels": {
+            "nvfp4_quantize_act": {"us": 1e3 * q_mean, "GB/s": q_gbs, "frac_hbm": q_gbs / hbm,
+                                   "bytes": q_bytes, "hbm_peak": hbm},
+            "nvfp4_gemm": {"us": 1e3 * g_mean, "TFLOP/s": gemm_tflops,
+                           "frac_fp4": gemm_tflops / fp4_peak,
+                           "frac_fp4_datasheet": gemm_tflops / 9000.0},
+        },
+        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
+        "gpu_launches": 2 * args.steps,
+        "clocks": sampler.summary(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, fl, cores = cpu_oracle_sample(wl, args.cpu_rows, A_cpu)
+        line["cpu_baseline"] = {
+            "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"{args.cpu_rows} of {M} rows of A: quantize + fp64 GEMM against the "
+                      f"full weight ({dt:.1f} s)"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del gq, gg
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_bsp(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,234 @@
+"""Python binding of ``libbsp.so``: the NVFP4 / fp8r quantized linear on B200.
+
+Argument marshalling only.  Every step of the path runs in the library's CUDA
+kernels; torch supplies device memory and the current stream.  There is no CPU
+fallback: importing works without a GPU (so the ABI can be inspected), but every
+compute call needs the built library and a compute-capability-10.0 device, and
+raises ``BSPError`` otherwise.
+
+The C entry points and their semantics are declared in ``include/bsp.h``; the
+functions here carry the same names.  Formats ("BFL (fp8r / nvfp4)", Diffusers
+quantization doc, format bullets): nvfp4 = packed E2M1 codes, E4M3 scale per 16
+elements, fp32 global scales; fp8r = E4M3 values with an fp32 scale per row.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "BSPError", "SF_LINEAR", "SF_MMA", "lib", "library_path",
+    "nvfp4_quantize_act", "nvfp4_gemm", "fp8r_quantize_rows", "fp8r_gemm",
+    "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
+    "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
+    "bsp_testing_gemm_stall",
+]
+
+SF_LINEAR = 0
+SF_MMA = 1
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_HERE, "libbsp.so")
+
+_c_i64 = ctypes.c_int64
+_c_int = ctypes.c_int
+_c_vp = ctypes.c_void_p
+
+_SIGS = {
+    "nvfp4_quantize_act": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_int, _c_vp], _c_int),
+    "nvfp4_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
+                    _c_i64, _c_vp], _c_int),
+    "fp8r_quantize_rows": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp], _c_int),
+    "fp8r_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp],
+                  _c_int),
+    "nvfp4_global_scale": ([_c_vp, _c_i64, _c_vp, _c_vp], _c_int),
+    "nvfp4_sf_convert": ([_c_vp, _c_vp, _c_i64, _c_i64, _c_int, _c_int, _c_vp], _c_int),
+    "nvfp4_sf_bytes": ([_c_i64, _c_i64, _c_int], _c_i64),
+    "bsp_last_device_status": ([_c_vp], _c_int),
+    "bsp_set_wait_limit_ms": ([_c_i64], _c_i64),
+    "bsp_status_string": ([_c_int], ctypes.c_char_p),
+    "bsp_version": ([], _c_int),
+    "bsp_testing_gemm_stall": ([_c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64,
+                                _c_i64, _c_i64, _c_i64, _c_i64, _c_vp], _c_int),
+}
+
+_lib = None
+
+
+class BSPError(RuntimeError):
+    """A libbsp call returned a negative bsp_status."""
+
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {status_name(status)} ({status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libbsp.so`` (raises if it has not been built: there is no fallback)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(library_path):
+            raise BSPError("load", -5) from FileNotFoundError(
+                f"{library_path} is missing; build it with "
+                "`python -m block_scaled_precision_act_b200.build` (or __graft_entry__.build())")
+        L = ctypes.CDLL(library_path)
+        for name, (argtypes, restype) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.argtypes = argtypes
+            fn.restype = restype
+        _lib = L
+    return _lib
+
+
+def status_name(status: int) -> str:
+    names = {0: "BSP_OK", -1: "BSP_ERR_INVALID_ARG", -2: "BSP_ERR_UNSUPPORTED_SHAPE",
+             -3: "BSP_ERR_MISALIGNED", -4: "BSP_ERR_UNSUPPORTED_DEVICE", -5: "BSP_ERR_CUDA",
+             -6: "BSP_ERR_TIMEOUT"}
+    return names.get(status, "BSP_ERR_UNKNOWN")
+
+
+def _check(fn: str, st: int) -> None:
+    if st != 0:
+        raise BSPError(fn, st)
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if not t.is_cuda:
+        raise BSPError("argument check (tensor not on a CUDA device)", -1)
+    if not t.is_contiguous():
+        raise BSPError("argument check (tensor not contiguous)", -1)
+    return t.data_ptr()
+
+
+def _stream(stream):
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, torch.cuda.Stream):
+        return stream.cuda_stream
+    return int(stream)
+
+
+def _dtype(t, dt, what):
+    if t.dtype != dt:
+        raise TypeError(f"{what} must be {dt}, got {t.dtype}")
+
+
+# ------------------------------------------------------------------ entry points
+def nvfp4_sf_bytes(rows: int, K: int, layout: int = SF_MMA) -> int:
+    n = lib().nvfp4_sf_bytes(rows, K, layout)
+    if n < 0:
+        raise BSPError("nvfp4_sf_bytes", int(n))
+    return int(n)
+
+
+def nvfp4_quantize_act(x: torch.Tensor, global_scale: torch.Tensor, codes=None, scales=None,
+                       layout: int = SF_MMA, stream=None):
+    """bf16 [M, K] -> (codes uint8 [M, K/2], block scales uint8 in `layout`)."""
+    _dtype(x, torch.bfloat16, "x")
+    _dtype(global_scale, torch.float32, "global_scale")
+    M, K = x.shape
+    if codes is None:
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
+    if scales is None:
+        scales = torch.empty((max(nvfp4_sf_bytes(M, K, layout), 0),), dtype=torch.uint8,
+                             device=x.device)
+    _check("nvfp4_quantize_act",
+           lib().nvfp4_quantize_act(_ptr(x), M, K, _ptr(global_scale), _ptr(codes),
+                                    _ptr(scales), layout, _stream(stream)))
+    return codes, scales
+
+
+def nvfp4_gemm(a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias=None, out=None,
+               stream=None):
+    """Y[M, N] bf16 = (a_global*w_global) * (A_q . W_q^T) (+ bias); scales in SF_MMA layout."""
+    M, K2 = a_codes.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] != K2:
+        raise BSPError("nvfp4_gemm (K mismatch)", -1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _check("nvfp4_gemm",
+           lib().nvfp4_gemm(_ptr(a_codes), _ptr(a_sf), _ptr(a_global), _ptr(w_codes),
+                            _ptr(w_sf), _ptr(w_global), _ptr(bias), _ptr(out), M, N, 2 * K2,
+                            _stream(stream)))
+    return out
+
+
+def fp8r_quantize_rows(x: torch.Tensor, q=None, row_scale=None, stream=None):
+    """bf16 [M, K] -> (E4M3 codes uint8 [M, K], fp32 row scales [M])."""
+    _dtype(x, torch.bfloat16, "x")
+    M, K = x.shape
+    if q is None:
+        q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
+    if row_scale is None:
+        row_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _check("fp8r_quantize_rows",
+           lib().fp8r_quantize_rows(_ptr(x), M, K, _ptr(q), _ptr(row_scale), _stream(stream)))
+    return q, row_scale
+
+
+def fp8r_gemm(a_q, a_row_scale, w_q, w_row_scale, bias=None, out=None, stream=None):
+    """Y[M, N] bf16 = (A_q . W_q^T) * sA[m] * sW[n] (+ bias)."""
+    M, K = a_q.shape
+    N = w_q.shape[0]
+    if w_q.shape[1] != K:
+        raise BSPError("fp8r_gemm (K mismatch)", -1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    _check("fp8r_gemm",
+           lib().fp8r_gemm(_ptr(a_q), _ptr(a_row_scale), _ptr(w_q), _ptr(w_row_scale),
+                           _ptr(bias), _ptr(out), M, N, K, _stream(stream)))
+    return out
+
+
+def nvfp4_global_scale(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+    """fp32 [1] = amax(x) / (448*6), computed on the device."""
+    _dtype(x, torch.bfloat16, "x")
+    if out is None:
+        out = torch.empty((1,), dtype=torch.float32, device=x.device)
+    _check("nvfp4_global_scale",
+           lib().nvfp4_global_scale(_ptr(x), x.numel(), _ptr(out), _stream(stream)))
+    return out
+
+
+def nvfp4_sf_convert(src, rows: int, K: int, from_layout: int, to_layout: int, dst=None,
+                     stream=None):
+    if dst is None:
+        dst = torch.empty((nvfp4_sf_bytes(rows, K, to_layout),), dtype=torch.uint8,
+                          device=src.device)
+    _check("nvfp4_sf_convert",
+           lib().nvfp4_sf_convert(_ptr(src), _ptr(dst), rows, K, from_layout, to_layout,
+                                  _stream(stream)))
+    return dst
+
+
+def bsp_last_device_status(stream=None) -> int:
+    return int(lib().bsp_last_device_status(_stream(stream)))
+
+
+def bsp_set_wait_limit_ms(ms: int) -> int:
+    return int(lib().bsp_set_wait_limit_ms(ms))
+
+
+def bsp_status_string(status: int) -> str:
+    return lib().bsp_status_string(status).decode()
+
+
+def bsp_version() -> int:
+    return int(lib().bsp_version())
+
+
+def bsp_testing_gemm_stall(scheme: int, a, a_sf, a_scale, w, w_sf, w_scale, out, K: int,
+                           stop_after_stages: int, wait_limit_ms: int, stream=None) -> int:
+    """Test hook (include/bsp_testing.h): returns the launch status, not the device status."""
+    M = a.shape[0]
+    N = w.shape[0]
+    return int(lib().bsp_testing_gemm_stall(scheme, _ptr(a), _ptr(a_sf), _ptr(a_scale), _ptr(w),
+                                            _ptr(w_sf), _ptr(w_scale), _ptr(out), M, N, K,
+                                            stop_after_stages, wait_limit_ms, _stream(stream)))

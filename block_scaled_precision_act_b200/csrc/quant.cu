@@ -1,0 +1,391 @@
+// quant.cu -- the run-time quantizers: NVFP4 block-16 activation quantizer, fp8r
+// per-row quantizer, the global-scale (amax) helper and the scale re-layout helper.
+//
+// "BFL (fp8r / nvfp4)" (Diffusers quantization doc): nvfp4 format bullet (E2M1
+// packed two per byte, E4M3 scale per 16-element block, fp32 global scales) and
+// fp8r bullet (activations quantized to E4M3 per row at run time); Kernels table
+// (the nvfp4 path quantizes activations before the FP4 GEMM).
+//
+// Both quantizers are HBM-bound streaming kernels: 128-bit coalesced loads of bf16,
+// warp-shuffle reductions, and coalesced stores of the packed codes.  The
+// arithmetic is fixed step by step (IEEE binary32, round to nearest even, no FTZ,
+// no fast-math) so that codes and scale bytes are bit-identical to the definition:
+//   nvfp4: t = 6g ; s = t > 0 ? amax/t : 0 ; sb = E4M3(s) ; d = dec(sb)*g ;
+//          d == 0 -> codes 0 ; else code = E2M1(x * min(1/d, FLT_MAX))
+//   fp8r : s = amax/448 ; s == 0 -> codes 0 ; else q = E4M3(x * min(1/s, FLT_MAX))
+#include <cfloat>
+#include <cstdint>
+
+#include "bsp_internal.h"
+#include "bsp_ptx.cuh"
+
+namespace bsp {
+namespace {
+
+constexpr int kQuantThreads = 256;
+constexpr int kQuantUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p)
+{
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void unpack8(const uint4& v, float (&f)[8])
+{
+    f[0] = bf16lo_to_f32(v.x); f[1] = bf16hi_to_f32(v.x);
+    f[2] = bf16lo_to_f32(v.y); f[3] = bf16hi_to_f32(v.y);
+    f[4] = bf16lo_to_f32(v.z); f[5] = bf16hi_to_f32(v.z);
+    f[6] = bf16lo_to_f32(v.w); f[7] = bf16hi_to_f32(v.w);
+}
+
+__device__ __forceinline__ int64_t sf_mma_offset(int64_t row, int64_t kb, int64_t kb4)
+{
+    return ((row >> 7) * kb4 + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 +
+           (kb & 3);
+}
+
+// One warp-iteration handles 32*U consecutive "octets" (8 bf16 each); lanes 2j and
+// 2j+1 of an iteration hold the two halves of one 16-element block.
+template <int LAYOUT>
+__global__ void __launch_bounds__(kQuantThreads)
+    nvfp4_quant_kernel(const uint4* __restrict__ x, int64_t total_oct, int64_t oct_per_row,
+                       const float* __restrict__ gptr, uint32_t* __restrict__ codes,
+                       uint8_t* __restrict__ scales)
+{
+    const float g = __ldg(gptr);
+    const float t = __fmul_rn(6.0f, g);
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kQuantThreads) >> 5;
+    const int64_t nb_row = oct_per_row >> 1;        // blocks per row = K/16
+    const int64_t kb4 = (nb_row + 3) >> 2;          // MMA column tiles
+
+    for (int64_t base = warp * 32 * kQuantUnroll; base < total_oct;
+         base += nwarps * 32 * kQuantUnroll) {
+        uint4 v[kQuantUnroll];
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t o = base + u * 32 + lane;
+            v[u] = (o < total_oct) ? ld_stream(x + o) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kQuantUnroll; ++u) {
+            const int64_t o = base + u * 32 + lane;
+            float f[8];
+            unpack8(v[u], f);
+            float amax = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
+            const float s = (t > 0.0f) ? __fdiv_rn(amax, t) : 0.0f;
+            const uint32_t sb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
+            const float d = __fmul_rn(e4m3_to_f32(sb), g);
+            uint32_t word = 0;
+            if (d != 0.0f) {
+                const float r = fminf(__frcp_rn(d), FLT_MAX);
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[i], r);
+                word = cvt_e2m1x8(y);
+            }
+            if (LAYOUT == BSP_SF_LINEAR) {
+                if (o < total_oct) {
+                    codes[o] = word;
+                    if ((lane & 1) == 0) scales[o >> 1] = static_cast<uint8_t>(sb);
+                }
+            } else {
+                // gather the 4 scales of blocks kb..kb+3 (kb % 4 == 0) into lane 8i
+                const uint32_t s1 = __shfl_down_sync(0xffffffffu, sb, 2);
+                const uint32_t s2 = __shfl_down_sync(0xffffffffu, sb, 4);
+                const uint32_t s3 = __shfl_down_sync(0xffffffffu, sb, 6);
+                if (o < total_oct) {
+                    codes[o] = word;
+                    if ((lane & 7) == 0) {
+                        const int64_t row = o / oct_per_row;
+                        const int64_t kb = (o - row * oct_per_row) >> 1;
+                        const uint32_t w4 = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+                        *reinterpret_cast<uint32_t*>(scales + sf_mma_offset(row, kb, kb4)) = w4;
+                    }
+                }
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------- fp8r
+constexpr int kRowThreads = 128;
+
+__device__ __forceinline__ float block_max_128(float v, float* red)
+{
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+    __syncthreads();
+    v = fmaxf(fmaxf(red[0], red[1]), fmaxf(red[2], red[3]));
+    return v;
+}
+
+__device__ __forceinline__ uint2 quant8_e4m3(const float (&f)[8], float r)
+{
+    uint2 q;
+    q.x = cvt_e4m3x2(__fmul_rn(f[0], r), __fmul_rn(f[1], r)) |
+          (cvt_e4m3x2(__fmul_rn(f[2], r), __fmul_rn(f[3], r)) << 16);
+    q.y = cvt_e4m3x2(__fmul_rn(f[4], r), __fmul_rn(f[5], r)) |
+          (cvt_e4m3x2(__fmul_rn(f[6], r), __fmul_rn(f[7], r)) << 16);
+    return q;
+}
+
+// One CTA per row; the row is held in registers (CPT chunks of 8 per thread).
+template <int CPT>
+__global__ void __launch_bounds__(kRowThreads)
+    fp8r_quant_kernel(const uint4* __restrict__ x, int64_t K8, uint2* __restrict__ q,
+                      float* __restrict__ row_scale)
+{
+    __shared__ float red[4];
+    const int64_t row = blockIdx.x;
+    const uint4* xr = x + row * K8;
+    uint2* qr = q + row * K8;
+    uint4 v[CPT];
+    float amax = 0.0f;
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int64_t i = threadIdx.x + c * kRowThreads;
+        v[c] = (i < K8) ? ld_stream(xr + i) : make_uint4(0, 0, 0, 0);
+        float f[8];
+        unpack8(v[c], f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    }
+    amax = block_max_128(amax, red);
+    const float s = __fdiv_rn(amax, 448.0f);
+    if (threadIdx.x == 0) row_scale[row] = s;
+    const float r = (s == 0.0f) ? 0.0f : fminf(__frcp_rn(s), FLT_MAX);
+#pragma unroll
+    for (int c = 0; c < CPT; ++c) {
+        const int64_t i = threadIdx.x + c * kRowThreads;
+        if (i < K8) {
+            float f[8];
+            unpack8(v[c], f);
+            qr[i] = (s == 0.0f) ? make_uint2(0, 0) : quant8_e4m3(f, r);
+        }
+    }
+}
+
+// Rows too long to hold on chip: two passes over the row.
+__global__ void __launch_bounds__(kRowThreads)
+    fp8r_quant_long_kernel(const uint4* __restrict__ x, int64_t K8, uint2* __restrict__ q,
+                           float* __restrict__ row_scale)
+{
+    __shared__ float red[4];
+    const int64_t row = blockIdx.x;
+    const uint4* xr = x + row * K8;
+    uint2* qr = q + row * K8;
+    float amax = 0.0f;
+    for (int64_t i = threadIdx.x; i < K8; i += kRowThreads) {
+        float f[8];
+        unpack8(ld_stream(xr + i), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) amax = fmaxf(amax, fabsf(f[e]));
+    }
+    amax = block_max_128(amax, red);
+    const float s = __fdiv_rn(amax, 448.0f);
+    if (threadIdx.x == 0) row_scale[row] = s;
+    const float r = (s == 0.0f) ? 0.0f : fminf(__frcp_rn(s), FLT_MAX);
+    for (int64_t i = threadIdx.x; i < K8; i += kRowThreads) {
+        float f[8];
+        unpack8(ld_stream(xr + i), f);
+        qr[i] = (s == 0.0f) ? make_uint2(0, 0) : quant8_e4m3(f, r);
+    }
+}
+
+// ---------------------------------------------------------------- global scale
+__global__ void __launch_bounds__(256)
+    amax_kernel(const uint4* __restrict__ x, int64_t n8, unsigned int* __restrict__ out)
+{
+    __shared__ float red[8];
+    float m = 0.0f;
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n8;
+         i += static_cast<int64_t>(gridDim.x) * 256) {
+        float f[8];
+        unpack8(ld_stream(x + i), f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float b = red[0];
+        for (int w = 1; w < 8; ++w) b = fmaxf(b, red[w]);
+        // non-negative floats order like their bit patterns
+        atomicMax(out, __float_as_uint(b));
+    }
+}
+
+__global__ void global_scale_finalize_kernel(float* out)
+{
+    const float amax = __uint_as_float(*reinterpret_cast<unsigned int*>(out));
+    out[0] = __fdiv_rn(amax, 2688.0f);
+}
+
+// ---------------------------------------------------------------- scale re-layout
+__global__ void sf_to_mma_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                 int64_t rows, int64_t nb, int64_t kb4, int64_t dst_bytes)
+{
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < dst_bytes;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t tile = j >> 9, within = j & 511;
+        const int64_t rt = tile / kb4, ct = tile - rt * kb4;
+        const int64_t row = rt * 128 + ((within & 15) >> 2) * 32 + (within >> 4);
+        const int64_t kb = ct * 4 + (within & 3);
+        dst[j] = (row < rows && kb < nb) ? src[row * nb + kb] : 0;
+    }
+}
+
+__global__ void sf_to_linear_kernel(const uint8_t* __restrict__ src, uint8_t* __restrict__ dst,
+                                    int64_t rows, int64_t nb, int64_t kb4)
+{
+    const int64_t n = rows * nb;
+    for (int64_t j = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; j < n;
+         j += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t row = j / nb, kb = j - row * nb;
+        dst[j] = src[sf_mma_offset(row, kb, kb4)];
+    }
+}
+
+int grid_for(int64_t work_items, int per_block, int num_sms, int blocks_per_sm)
+{
+    int64_t need = (work_items + per_block - 1) / per_block;
+    int64_t cap = static_cast<int64_t>(num_sms) * blocks_per_sm;
+    if (need < 1) need = 1;
+    return static_cast<int>(need < cap ? need : cap);
+}
+
+}  // namespace
+}  // namespace bsp
+
+extern "C" {
+
+int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* global_scale,
+                       uint8_t* codes, uint8_t* scales, int layout, bsp_stream_t stream)
+{
+    using namespace bsp;
+    if (M < 0 || K <= 0 || (layout != BSP_SF_LINEAR && layout != BSP_SF_MMA))
+        return BSP_ERR_INVALID_ARG;
+    if (M == 0) return BSP_OK;
+    if (!x_bf16 || !global_scale || !codes || !scales) return BSP_ERR_INVALID_ARG;
+    if (K % 16 != 0 || (layout == BSP_SF_MMA && K % 64 != 0)) return BSP_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(codes) || !aligned16(scales) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+        return BSP_ERR_MISALIGNED;
+    int dev = 0, sms = 0;
+    int st = check_device(&dev, &sms);
+    if (st != BSP_OK) return st;
+    const int64_t total_oct = M * (K / 8);
+    const int grid = grid_for(total_oct, kQuantThreads * kQuantUnroll, sms, 8);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (layout == BSP_SF_LINEAR)
+        nvfp4_quant_kernel<BSP_SF_LINEAR><<<grid, kQuantThreads, 0, s>>>(
+            static_cast<const uint4*>(x_bf16), total_oct, K / 8, global_scale,
+            reinterpret_cast<uint32_t*>(codes), scales);
+    else
+        nvfp4_quant_kernel<BSP_SF_MMA><<<grid, kQuantThreads, 0, s>>>(
+            static_cast<const uint4*>(x_bf16), total_oct, K / 8, global_scale,
+            reinterpret_cast<uint32_t*>(codes), scales);
+    return launch_status();
+}
+
+int fp8r_quantize_rows(const void* x_bf16, int64_t M, int64_t K, uint8_t* q_e4m3,
+                       float* row_scale, bsp_stream_t stream)
+{
+    using namespace bsp;
+    if (M < 0 || K <= 0) return BSP_ERR_INVALID_ARG;
+    if (M == 0) return BSP_OK;
+    if (!x_bf16 || !q_e4m3 || !row_scale) return BSP_ERR_INVALID_ARG;
+    if (K % 8 != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
+    if (M > 0x7FFFFFFF) return BSP_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || !aligned16(q_e4m3) || !aligned16(row_scale))
+        return BSP_ERR_MISALIGNED;
+    int st = check_device(nullptr, nullptr);
+    if (st != BSP_OK) return st;
+    const int64_t K8 = K / 8;
+    const int64_t cpt = (K8 + kRowThreads - 1) / kRowThreads;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const auto* xv = static_cast<const uint4*>(x_bf16);
+    auto* qv = reinterpret_cast<uint2*>(q_e4m3);
+    const dim3 grid(static_cast<unsigned>(M));
+    if (cpt <= 1)
+        fp8r_quant_kernel<1><<<grid, kRowThreads, 0, s>>>(xv, K8, qv, row_scale);
+    else if (cpt <= 2)
+        fp8r_quant_kernel<2><<<grid, kRowThreads, 0, s>>>(xv, K8, qv, row_scale);
+    else if (cpt <= 4)
+        fp8r_quant_kernel<4><<<grid, kRowThreads, 0, s>>>(xv, K8, qv, row_scale);
+    else if (cpt <= 8)
+        fp8r_quant_kernel<8><<<grid, kRowThreads, 0, s>>>(xv, K8, qv, row_scale);
+    else if (cpt <= 16)
+        fp8r_quant_kernel<16><<<grid, kRowThreads, 0, s>>>(xv, K8, qv, row_scale);
+    else
+        fp8r_quant_long_kernel<<<grid, kRowThreads, 0, s>>>(xv, K8, qv, row_scale);
+    return launch_status();
+}
+
+int nvfp4_global_scale(const void* x_bf16, int64_t n, float* global_scale_out,
+                       bsp_stream_t stream)
+{
+    using namespace bsp;
+    if (n < 0 || !x_bf16 || !global_scale_out) return BSP_ERR_INVALID_ARG;
+    if (n % 8 != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(x_bf16) || (reinterpret_cast<uintptr_t>(global_scale_out) & 3u))
+        return BSP_ERR_MISALIGNED;
+    int dev = 0, sms = 0;
+    int st = check_device(&dev, &sms);
+    if (st != BSP_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaMemsetAsync(global_scale_out, 0, sizeof(float), s) != cudaSuccess) {
+        cudaGetLastError();
+        return BSP_ERR_CUDA;
+    }
+    if (n > 0) {
+        const int grid = grid_for(n / 8, 256 * 4, sms, 4);
+        amax_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x_bf16), n / 8,
+                                         reinterpret_cast<unsigned int*>(global_scale_out));
+        st = launch_status();
+        if (st != BSP_OK) return st;
+    }
+    global_scale_finalize_kernel<<<1, 1, 0, s>>>(global_scale_out);
+    return launch_status();
+}
+
+int nvfp4_sf_convert(const uint8_t* src, uint8_t* dst, int64_t rows, int64_t K, int from,
+                     int to, bsp_stream_t stream)
+{
+    using namespace bsp;
+    if (rows < 0 || K <= 0) return BSP_ERR_INVALID_ARG;
+    if (rows == 0) return BSP_OK;
+    if (!src || !dst) return BSP_ERR_INVALID_ARG;
+    if ((from != BSP_SF_LINEAR && from != BSP_SF_MMA) || (to != BSP_SF_LINEAR && to != BSP_SF_MMA) ||
+        from == to)
+        return BSP_ERR_INVALID_ARG;
+    if (K % 64 != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
+    int dev = 0, sms = 0;
+    int st = check_device(&dev, &sms);
+    if (st != BSP_OK) return st;
+    const int64_t nb = K / 16, kb4 = (nb + 3) / 4;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (to == BSP_SF_MMA) {
+        const int64_t bytes = nvfp4_sf_bytes(rows, K, BSP_SF_MMA);
+        sf_to_mma_kernel<<<grid_for(bytes, 256, sms, 8), 256, 0, s>>>(src, dst, rows, nb, kb4,
+                                                                       bytes);
+    } else {
+        sf_to_linear_kernel<<<grid_for(rows * nb, 256, sms, 8), 256, 0, s>>>(src, dst, rows, nb,
+                                                                             kb4);
+    }
+    return launch_status();
+}
+
+}  // extern "C"

@@ -1,0 +1,178 @@
+/*
+ * bsp.h -- C ABI of libbsp.so: the block-scaled precision linear on B200 (sm_100a).
+ *
+ * The operation is the quantized linear layer Y = X * W^T (+ bias) of a
+ * rectified-flow image transformer in the two storage schemes defined on the
+ * "BFL (fp8r / nvfp4)" page (Diffusers quantization doc, format bullets):
+ *
+ *   nvfp4 (ModelOpt layout): `weight` packed E2M1, two values per byte;
+ *          `weight_scale` E4M3, one per block of 16 elements along K;
+ *          `weight_scale_2` fp32 global scale; `input_scale` fp32 calibrated
+ *          activation scale.
+ *   fp8r : `weight` E4M3 with one fp32 `weight_scale` per row; activations are
+ *          quantized to E4M3 per row at run time.
+ *
+ * The same page's "Kernels" table pairs each scheme with a fused path: for nvfp4,
+ * an activation quantizer followed by a block-scaled FP4 GEMM; for fp8r, a
+ * row-scaled FP8 GEMM.  These entry points are that pair of calls for each scheme.
+ *
+ * Conventions for every call
+ *   - All pointers are DEVICE pointers unless stated otherwise, owned by the caller;
+ *     the library allocates nothing and keeps no per-call state.  Every tensor is
+ *     contiguous row-major.  All work is enqueued asynchronously on `stream`
+ *     (NULL = the legacy default stream); nothing synchronises the host.
+ *   - Tensor pointers must be 16-byte aligned (BSP_ERR_MISALIGNED otherwise).
+ *   - Argument errors are detected on the host before any launch and returned as a
+ *     negative bsp_status; nothing is enqueued in that case.  A zero-sized problem
+ *     (M == 0, or N == 0 for a GEMM) returns BSP_OK and enqueues nothing; its
+ *     pointers may then be NULL.
+ *   - Launch failures return BSP_ERR_CUDA.  Faults found by the kernels themselves
+ *     (a bounded wait that ran out) are recorded in a per-device status word and
+ *     reported by bsp_last_device_status().
+ *   - Only compute capability 10.0 (B200, sm_100a) is supported
+ *     (BSP_ERR_UNSUPPORTED_DEVICE otherwise).  There is no fallback path.
+ *
+ * Number formats
+ *   E2M1: sign, 2 exponent bits (bias 1), 1 mantissa bit; magnitudes
+ *         {0, 0.5, 1, 1.5, 2, 3, 4, 6}.  Packed two per byte: element 2j in bits 0-3,
+ *         element 2j+1 in bits 4-7.
+ *   E4M3: the "fn" variant (bias 7, no infinities, max 448, 0x7F/0xFF are NaN).
+ *   bf16 in and out.  Rounding everywhere is to nearest, ties to even; encoders
+ *   saturate (E2M1 at +-6, E4M3 at +-448) and keep the sign.
+ *
+ * Scale-factor layouts for NVFP4 block scales (one E4M3 byte per 16 elements):
+ *   BSP_SF_LINEAR: [rows][K/16] row-major.
+ *   BSP_SF_MMA   : the tiled layout the tensor cores read.  Rows are grouped in
+ *                  tiles of 128 and block-columns in tiles of 4; tile (rt, ct) is
+ *                  512 contiguous bytes at offset (rt * ceil(K/64) + ct) * 512, and
+ *                  inside it row r, block-column c sits at
+ *                  (r % 32) * 16 + ((r / 32) % 4) * 4 + (c % 4).
+ *                  Its size is nvfp4_sf_bytes(rows, K, BSP_SF_MMA) (rows padded to
+ *                  a multiple of 128); padding bytes are never read for results.
+ */
+#ifndef BSP_H_
+#define BSP_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* bsp_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+    BSP_OK = 0,
+    BSP_ERR_INVALID_ARG = -1,       /* null pointer, bad enum, negative size        */
+    BSP_ERR_UNSUPPORTED_SHAPE = -2, /* a size outside the documented constraints    */
+    BSP_ERR_MISALIGNED = -3,        /* a tensor pointer not 16-byte aligned         */
+    BSP_ERR_UNSUPPORTED_DEVICE = -4,/* current device is not compute capability 10.0 */
+    BSP_ERR_CUDA = -5,              /* a CUDA runtime call or launch failed          */
+    BSP_ERR_TIMEOUT = -6            /* a kernel's bounded wait ran out (device side) */
+} bsp_status;
+
+typedef enum { BSP_SF_LINEAR = 0, BSP_SF_MMA = 1 } bsp_sf_layout;
+
+/*
+ * nvfp4_quantize_act -- NVFP4 activation quantizer ("BFL (fp8r / nvfp4)", Kernels
+ * table: the activations of an nvfp4 linear are quantized before the FP4 GEMM; the
+ * format bullet gives block 16, E4M3 block scales and the fp32 `input_scale`).
+ *
+ *   x_bf16        [M][K] bf16.
+ *   global_scale  device pointer to ONE fp32: the decode-side global scale g
+ *                 (`input_scale` for activations, `weight_scale_2` for weights).
+ *   codes         out [M][K/2] bytes, packed E2M1.
+ *   scales        out E4M3 block scales in `layout` (nvfp4_sf_bytes(M, K, layout)).
+ * Per block b of 16 elements along K (every step one IEEE binary32 operation):
+ *   s_b = amax_b / (6 g) (0 when 6 g is 0) ; scales[b] = E4M3(s_b) ; d = e4m3(scales[b]) * g ;
+ *   d == 0 -> all 16 codes 0 ; else code_i = E2M1(x_i * (1/d)), 1/d clamped to FLT_MAX.
+ * Constraints: K % 16 == 0; BSP_SF_MMA also needs K % 64 == 0.
+ */
+int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* global_scale,
+                       uint8_t* codes, uint8_t* scales, int layout, bsp_stream_t stream);
+
+/*
+ * nvfp4_gemm -- block-scaled FP4 GEMM with the dequantisation fused into the
+ * epilogue ("BFL (fp8r / nvfp4)", Kernels table: the nvfp4 fused GEMM).
+ *
+ *   a_codes [M][K/2], a_sf (BSP_SF_MMA, rows = M), a_global (device, 1 fp32 = input_scale)
+ *   w_codes [N][K/2], w_sf (BSP_SF_MMA, rows = N), w_global (device, 1 fp32 = weight_scale_2)
+ *   bias_bf16  [N] bf16 or NULL.
+ *   out_bf16   [M][N] bf16.
+ *   Y[m][n] = bf16( acc[m][n] * (a_global * w_global) + bias[n] ),
+ *   acc = sum_k e2m1(a)*e4m3(sa) * e2m1(w)*e4m3(sw), accumulated in fp32 on the
+ *   tensor cores.
+ * Constraints: K % 64 == 0, K >= 64; N % 8 == 0.  Any M >= 0.
+ */
+int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+               const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+               const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
+               bsp_stream_t stream);
+
+/*
+ * fp8r_quantize_rows -- per-row E4M3 quantizer ("BFL (fp8r / nvfp4)", fp8r bullet:
+ * activations are quantized to E4M3 per row at run time; weights use one fp32 scale
+ * per row).
+ *   x_bf16 [M][K] bf16 ; q_e4m3 out [M][K] ; row_scale out [M] fp32.
+ *   s_m = amax_m / 448 ; s_m == 0 -> q = 0 ; else q = E4M3(x * (1/s_m)), 1/s_m
+ *   clamped to FLT_MAX.
+ * Constraints: K % 8 == 0.
+ */
+int fp8r_quantize_rows(const void* x_bf16, int64_t M, int64_t K, uint8_t* q_e4m3,
+                       float* row_scale, bsp_stream_t stream);
+
+/*
+ * fp8r_gemm -- row-scaled FP8 GEMM ("BFL (fp8r / nvfp4)", Kernels table: the fp8r
+ * fused GEMM with per-row scales).
+ *   a_e4m3 [M][K], a_row_scale [M]; w_e4m3 [N][K], w_row_scale [N]; bias [N] or NULL.
+ *   Y[m][n] = bf16( (acc[m][n] * sA[m]) * sW[n] + bias[n] ), acc in fp32 on the
+ *   tensor cores.
+ * Constraints: K % 16 == 0, K >= 16; N % 8 == 0.  Any M >= 0.
+ */
+int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_e4m3,
+              const float* w_row_scale, const void* bias_bf16, void* out_bf16, int64_t M,
+              int64_t N, int64_t K, bsp_stream_t stream);
+
+/*
+ * nvfp4_global_scale -- g = amax(X) / (448 * 6) over n bf16 values, written to the
+ * device fp32 at `global_scale_out` (the nvfp4 `weight_scale_2` / `input_scale`
+ * convention: a decode-side multiplier that maps the largest block scale to the
+ * E4M3 maximum).  Enqueues a clear of the output, an atomic max over the input and a
+ * final divide; no scratch memory.  Constraints: n % 8 == 0.
+ */
+int nvfp4_global_scale(const void* x_bf16, int64_t n, float* global_scale_out,
+                       bsp_stream_t stream);
+
+/*
+ * nvfp4_sf_convert -- re-lay block scales between BSP_SF_LINEAR and BSP_SF_MMA
+ * (rows x K/16 bytes; padding of an MMA-layout destination is written as 0).
+ * Constraints: K % 64 == 0.  src and dst must not overlap.
+ */
+int nvfp4_sf_convert(const uint8_t* src, uint8_t* dst, int64_t rows, int64_t K, int from,
+                     int to, bsp_stream_t stream);
+
+/* Bytes of a scale array of `rows` x K/16 in `layout`; negative on bad arguments. */
+int64_t nvfp4_sf_bytes(int64_t rows, int64_t K, int layout);
+
+/*
+ * bsp_last_device_status -- synchronises `stream`, returns and clears the status
+ * word the kernels of the current device write (BSP_OK, or BSP_ERR_TIMEOUT when a
+ * bounded wait inside a GEMM ran out).  BSP_ERR_CUDA if the synchronisation fails.
+ */
+int bsp_last_device_status(bsp_stream_t stream);
+
+/* Bounded-wait limit of the GEMM kernels in milliseconds (default 2000, also set by
+ * the BSP_WAIT_LIMIT_MS environment variable at first use).  Returns the old value. */
+int64_t bsp_set_wait_limit_ms(int64_t ms);
+
+/* Human-readable name of a bsp_status value. */
+const char* bsp_status_string(int status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int bsp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSP_H_ */

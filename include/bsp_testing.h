@@ -1,0 +1,38 @@
+/*
+ * bsp_testing.h -- test hooks of libbsp.so (not part of the compute path).
+ *
+ * The pages describe no failure handling; these hooks exist so the bounded waits
+ * inside the GEMM kernels can be exercised without faulting or hanging a GPU.
+ */
+#ifndef BSP_TESTING_H_
+#define BSP_TESTING_H_
+
+#include <stdint.h>
+
+#include "bsp.h"
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/*
+ * bsp_testing_gemm_stall -- runs the nvfp4 (scheme 1) or fp8r (scheme 0) GEMM with
+ * the producer stopping after `stop_after_stages` K-stages, so the MMA thread's
+ * wait on the next stage can never complete.  Every wait in the kernel is bounded
+ * by `wait_limit_ms` (1..10000); the kernel then records BSP_ERR_TIMEOUT in the
+ * device status word, waits for the copies and MMAs it already issued, frees its
+ * tensor memory and exits, leaving the context usable.  Arguments are those of
+ * nvfp4_gemm / fp8r_gemm (a_sf / w_sf ignored for fp8r; no bias).  The output is
+ * left partially written.  Read the outcome with bsp_last_device_status().
+ */
+int bsp_testing_gemm_stall(int scheme, const uint8_t* a, const uint8_t* a_sf,
+                           const float* a_scale, const uint8_t* w, const uint8_t* w_sf,
+                           const float* w_scale, void* out_bf16, int64_t M, int64_t N,
+                           int64_t K, int64_t stop_after_stages, int64_t wait_limit_ms,
+                           bsp_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BSP_TESTING_H_ */
