@@ -23,7 +23,7 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_gemm", "fp8r_quantize_rows", "fp8r_gemm",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
-    "bsp_testing_gemm_stall",
+    "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel",
 ]
 
 SF_LINEAR = 0
@@ -50,6 +50,7 @@ _SIGS = {
     "bsp_set_wait_limit_ms": ([_c_i64], _c_i64),
     "bsp_status_string": ([_c_int], ctypes.c_char_p),
     "bsp_version": ([], _c_int),
+    "bsp_testing_set_gemm_kernel": ([_c_int], _c_int),
     "bsp_testing_gemm_stall": ([_c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64,
                                 _c_i64, _c_i64, _c_i64, _c_i64, _c_vp], _c_int),
 }
@@ -232,3 +233,11 @@ def bsp_testing_gemm_stall(scheme: int, a, a_sf, a_scale, w, w_sf, w_scale, out,
     return int(lib().bsp_testing_gemm_stall(scheme, _ptr(a), _ptr(a_sf), _ptr(a_scale), _ptr(w),
                                             _ptr(w_sf), _ptr(w_scale), _ptr(out), M, N, K,
                                             stop_after_stages, wait_limit_ms, _stream(stream)))
+
+
+def bsp_testing_set_gemm_kernel(choice: int) -> int:
+    """Test hook: 0 = automatic, 1 = CTA-pair kernel, 2 = single-CTA kernel."""
+    old = int(lib().bsp_testing_set_gemm_kernel(choice))
+    if old < 0:
+        raise BSPError("bsp_testing_set_gemm_kernel", old)
+    return old

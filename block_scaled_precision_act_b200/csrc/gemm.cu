@@ -22,8 +22,11 @@
 //               32-lane quadrant), scales, bias, bf16 rounding, stores.
 // Tiles are 128 x BN; tile t of a CTA is blockIdx.x + i*gridDim.x, M-fastest so that
 // neighbouring CTAs share the weight tile.  No cluster multicast is used anywhere.
+#include <atomic>
 #include <cfloat>
 #include <cstdint>
+#include <cstdlib>
+#include <cstring>
 #include <mutex>
 
 #include <cuda.h>
@@ -342,6 +345,381 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 1) tmem_dealloc(tbase, kTmemCols);
 }
 
+// ---------------------------------------------------------------- CTA-pair kernel
+// Two CTAs of a cluster compute one 256 x 256 tile with tcgen05 cta_group::2: CTA r
+// loads rows [128r, 128r+128) of the A tile and rows [128r, 128r+128) of the B tile
+// (its half of N); the MMA thread of CTA 0 issues one 256x256xK MMA that reads both
+// CTAs' shared memory and writes each CTA's 128 x 256 accumulator into that CTA's
+// TMEM.  Both CTAs fetch the scale factors of all 256 B rows (no multicast).
+//
+// Roles (13 warps per CTA):
+//   warp 0       TMA producer (both CTAs) into a ring of K-stages of 128 bytes per row;
+//   warp 1       TMEM allocation; in CTA 0 one thread issues the MMAs;
+//   warps 2..4   (CTA 0, nvfp4) scale-factor copies smem -> TMEM, one chunk kind per
+//                warp (A, B rows 0-127, B rows 128-255).  A tcgen05.cp costs about as
+//                much issue time as an MMA K-step, so issuing them from the MMA thread
+//                would serialise them with the MMAs; from other warps they overlap.
+//                The copies go into one of two TMEM scale buffers (stage parity).
+//   warps 5..12  epilogue, two warps per 32-lane TMEM quadrant, 32-column subtiles.
+// TMEM columns: accumulator 0 = [0, 256), accumulator 1 = [160, 416) (they share 96
+// columns), scale buffers at [416, 464) and [464, 512).  The epilogue drains the shared
+// columns first and then releases the accumulator, so the next tile's MMAs overlap the
+// rest of the epilogue.  Output goes through a 64-byte-swizzled smem slab per warp and
+// a TMA store.
+template <bool NVF4>
+struct PairCfg {
+    static constexpr int STAGES = NVF4 ? 5 : 6;
+    static constexpr int THREADS = 13 * 32;
+    static constexpr int A_BYTES = 128 * kBKB;
+    static constexpr int B_BYTES = 128 * kBKB;
+    static constexpr int SFA_BYTES = NVF4 ? 2048 : 0;
+    static constexpr int SFB_BYTES = NVF4 ? 4096 : 0;
+    static constexpr int K_STAGE = NVF4 ? 256 : 128;
+    static constexpr int K_MMA = NVF4 ? 64 : 32;
+    static constexpr int STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
+    static constexpr int EPI_WARPS = 8;
+    static constexpr int EPI_SLAB = 32 * 64;           // one warp's 32 rows x 32 bf16
+    static constexpr int OFF_B = STAGES * A_BYTES;
+    static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+    static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+    static constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_BYTES;
+    static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * 2 * EPI_SLAB;
+    static constexpr int NUM_BARS = 2 * STAGES + 4 + 4;
+    static constexpr int SMEM_BYTES = 1024 + OFF_BAR + NUM_BARS * 8 + 16;
+    static constexpr int ACC_STRIDE = 160;
+    static constexpr int SF_COL0 = 416;                // two buffers of 48 columns
+    static constexpr int SF_BUF = 48;                  // SFA 16 + SFB 32 per K-stage
+    static constexpr uint32_t IDESC = NVF4 ? idesc_nvf4(256, 256) : idesc_e4m3(256, 256);
+    static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+    static_assert(OFF_EPI % 1024 == 0, "epilogue slabs must be 1024-byte aligned");
+    static_assert(SF_COL0 + 2 * SF_BUF <= 512 && ACC_STRIDE + 256 <= SF_COL0, "TMEM budget");
+};
+
+template <bool NVF4>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREADS, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                     const __grid_constant__ CUtensorMap tmB,
+                     const __grid_constant__ CUtensorMap tmSFA,
+                     const __grid_constant__ CUtensorMap tmSFB,
+                     const __grid_constant__ CUtensorMap tmY, const GemmArgs args)
+{
+    using C = PairCfg<NVF4>;
+    constexpr int STAGES = C::STAGES;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + C::OFF_B;
+    uint8_t* sSFA = smem + C::OFF_SFA;
+    uint8_t* sSFB = smem + C::OFF_SFB;
+    uint8_t* sEpi = smem + C::OFF_EPI;
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+    uint64_t* empty = full + STAGES;
+    uint64_t* sf_full = empty + STAGES;     // [2]
+    uint64_t* sf_empty = sf_full + 2;       // [2]
+    uint64_t* acc_full = sf_empty + 2;
+    uint64_t* acc_empty = acc_full + 1;
+    uint64_t* fin = acc_empty + 1;
+    uint64_t* cp_fin = fin + 1;             // copy warps' last commits
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(cp_fin + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1;
+    const int npairs = gridDim.x >> 1;
+    const int M = args.M, N = args.N, K = args.K;
+    const int num_m = (M + 255) / 256;
+    const int num_n = (N + 255) / 256;
+    const int num_tiles = num_m * num_n;
+    const int num_kt = (K + C::K_STAGE - 1) / C::K_STAGE;
+    const int kb4 = (K / 16 + 3) / 4;
+
+    if (warp == 0 && lane == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(full + s, 1);
+            mbar_init(empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(sf_full + b, 3);      // one commit per copy warp
+            mbar_init(sf_empty + b, 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(acc_empty, 2 * C::EPI_WARPS);   // epilogue warps of both CTAs
+        mbar_init(fin, 1);
+        mbar_init(cp_fin, 3);
+        *abort_flag = 0;
+        fence_mbar_init();
+        prefetch_tmap(&tmA);
+        prefetch_tmap(&tmB);
+        prefetch_tmap(&tmY);
+        if constexpr (NVF4) {
+            prefetch_tmap(&tmSFA);
+            prefetch_tmap(&tmSFB);
+        }
+    }
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_holder, kTmemCols);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    const uint32_t tbase = *tmem_holder;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int64_t it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+                const int mt = tile % num_m, nt = tile / num_m;
+                const int a_row = mt * 256 + static_cast<int>(rank) * 128;
+                const int b_row = nt * 256 + static_cast<int>(rank) * 128;
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    if (it == args.debug_stop_iter) { ok = false; break; }
+                    const int s = static_cast<int>(it % STAGES);
+                    const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
+                    if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.wait_ns, args.status, 11)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t bar0 = mapa_shared(smem_u32(full + s), 0);
+                    if (rank == 0) mbar_arrive_expect_tx(full + s, 2 * C::STAGE_TX);
+                    tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar0, kt * kBKB, a_row);
+                    tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar0, kt * kBKB, b_row);
+                    if constexpr (NVF4) {
+                        // scale chunks are 32 rows of 16 bytes; a stage needs 4 chunks
+                        const int ya = ((a_row / 128) * kb4 + 4 * kt) * 32;
+                        tma_load_2d_pair(sSFA + s * C::SFA_BYTES, &tmSFA, bar0, 0, ya);
+                        for (int c = 0; c < 2; ++c) {
+                            const int yb = ((nt * 2 + c) * kb4 + 4 * kt) * 32;
+                            tma_load_2d_pair(sSFB + s * C::SFB_BYTES + c * 2048, &tmSFB, bar0, 0,
+                                             yb);
+                        }
+                    }
+                    ++it;
+                }
+            }
+            if (rank == 0) {
+                for (int64_t i = (it > STAGES ? it - STAGES : 0); i < it; ++i)
+                    drain_wait(full + (i % STAGES), static_cast<uint32_t>((i / STAGES) & 1),
+                               args.wait_ns, args.status);
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (CTA 0)
+        if (lane == 0 && rank == 0) {
+            int64_t it = 0;
+            int acc_it = 0;
+            bool ok = true;
+            for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+                if (acc_it > 0 &&
+                    !mbar_wait(acc_empty, static_cast<uint32_t>((acc_it - 1) & 1), abort_flag,
+                               args.wait_ns, args.status, 12))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tbase + static_cast<uint32_t>((acc_it & 1) * C::ACC_STRIDE);
+                for (int kt = 0; kt < num_kt; ++kt) {
+                    const int s = static_cast<int>(it % STAGES);
+                    const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
+                    const int b = static_cast<int>(it & 1);
+                    if (!mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status, 13)) {
+                        ok = false;
+                        break;
+                    }
+                    int nk;
+                    if constexpr (NVF4) {
+                        if (!mbar_wait(sf_full + b, static_cast<uint32_t>((it >> 1) & 1), abort_flag,
+                                       args.wait_ns, args.status, 15)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        nk = min(4, K / 64 - 4 * kt);
+                    } else {
+                        nk = min(4, (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
+                    }
+                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + s * C::A_BYTES));
+                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * C::B_BYTES));
+                    const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
+                    for (int k = 0; k < nk; ++k) {
+                        const uint32_t acc = (kt > 0 || k > 0) ? 1u : 0u;
+                        if constexpr (NVF4)
+                            mma_nvf4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::IDESC, sf + k * 4,
+                                          sf + 16 + k * 8, acc);
+                        else
+                            mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::IDESC, acc);
+                    }
+                    tc_commit_pair(empty + s, 0x3);
+                    if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
+                    ++it;
+                }
+                if (!ok) break;
+                tc_commit_pair(acc_full, 0x3);
+                ++acc_it;
+            }
+        }
+    } else if (warp <= 4) {
+        // ------------------------------------------------------------ scale copies (CTA 0)
+        if constexpr (NVF4) {
+            if (lane == 0 && rank == 0) {
+                const int which = warp - 2;          // 0: SFA, 1: SFB rows 0-127, 2: rows 128-255
+                int64_t it = 0;
+                bool ok = true;
+                for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
+                    for (int kt = 0; kt < num_kt; ++kt) {
+                        const int s = static_cast<int>(it % STAGES);
+                        const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
+                        const int b = static_cast<int>(it & 1);
+                        if (!mbar_wait(sf_empty + b, static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                                       abort_flag, args.wait_ns, args.status, 16) ||
+                            !mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status, 17)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        const int nk = min(4, K / 64 - 4 * kt);
+                        const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
+                        for (int kb = 0; kb < nk; ++kb) {
+                            if (which == 0)
+                                tmem_cp_32x128b_x4_pair(
+                                    sf + kb * 4,
+                                    sdesc_sf_block(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512)));
+                            else
+                                tmem_cp_32x128b_x4_pair(
+                                    sf + 16 + kb * 8 + (which - 1) * 4,
+                                    sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES +
+                                                            (which - 1) * 2048 + kb * 512)));
+                        }
+                        tc_commit_pair(sf_full + b, 0x1);
+                        ++it;
+                    }
+                }
+                tc_commit_pair(cp_fin, 0x1);     // lets the teardown wait for every copy
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - 5;              // 0..7
+        const int q = warp & 3;               // TMEM lane quadrant this warp may access
+        const int h = ew >> 2;                // which half of the subtiles
+        const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
+        uint8_t* slab0 = sEpi + ew * 2 * C::EPI_SLAB;
+        float alpha = 0.0f;
+        if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
+        int acc_it = 0;
+        int buf = 0;
+        int committed = 0;               // bulk-store groups this warp committed
+        int last_group[2] = {-1, -1};    // group that last read each slab
+        for (int tile = pair; tile < num_tiles; tile += npairs) {
+            const int mt = tile % num_m, nt = tile / num_m;
+            const bool ok = mbar_wait(acc_full, static_cast<uint32_t>(acc_it & 1), abort_flag,
+                                      args.wait_ns, args.status, 14);
+            if (!__all_sync(0xffffffffu, ok)) break;   // also reconverges the warp
+            tc_fence_after();
+            const int sacc = acc_it & 1;
+            const int wrow = mt * 256 + static_cast<int>(rank) * 128 + q * 32;   // warp's first row
+            const int m = wrow + lane;
+            float sa = 0.0f;
+            if constexpr (!NVF4) sa = (m < M) ? __ldg(args.a_scale + m) : 0.0f;
+            const uint32_t tq = tbase + (static_cast<uint32_t>(q * 32) << 16) +
+                                static_cast<uint32_t>(sacc * C::ACC_STRIDE);
+            // subtiles of 32 columns; the 3 shared with the other accumulator come first
+            // (columns 160..255 of accumulator 0, columns 0..95 of accumulator 1)
+#pragma unroll 1
+            for (int idx = 0; idx < 4; ++idx) {
+                const int ord = 2 * idx + h;                        // 0..7
+                const int j = sacc == 0 ? (ord + 5) & 7 : ord;
+                uint32_t r[32];
+                tmem_ld_x32(tq + j * 32, r);
+                tmem_ld_wait();
+                // the shared subtiles are ord 0, 1, 2: half 0 holds two, half 1 one
+                if ((h == 0 && idx == 1) || (h == 1 && idx == 0)) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cluster(acc_empty0);
+                }
+                const int n0 = nt * 256 + j * 32;
+                uint32_t packed[16];
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const int n = n0 + g * 8;
+                    float v[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[g * 8 + i]);
+                    if (n < N) {
+                        if constexpr (NVF4) {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], alpha);
+                        } else {
+                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(args.w_scale + n));
+                            const float4 w1 =
+                                __ldg(reinterpret_cast<const float4*>(args.w_scale + n + 4));
+                            const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], sa), sw[i]);
+                        }
+                        if (args.bias != nullptr) {
+                            const uint4 bb = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
+                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                v[2 * i] = __fadd_rn(v[2 * i], bf16lo_to_f32(bw[i]));
+                                v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16hi_to_f32(bw[i]));
+                            }
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) packed[g * 4 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                }
+                // the TMA store that last read this slab must be done reading it
+                if (lane == 0 && last_group[buf] >= 0) {
+                    if (committed - 1 - last_group[buf] == 0)
+                        bulk_wait_group_read<0>();
+                    else
+                        bulk_wait_group_read<1>();
+                }
+                __syncwarp();
+                uint8_t* slab = slab0 + buf * C::EPI_SLAB;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int pc = c ^ ((lane >> 1) & 3);           // 64-byte swizzle
+                    *reinterpret_cast<uint4*>(slab + lane * 64 + pc * 16) =
+                        make_uint4(packed[c * 4], packed[c * 4 + 1], packed[c * 4 + 2],
+                                   packed[c * 4 + 3]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (wrow < M && n0 < N) {
+                    if (lane == 0) {
+                        tma_store_2d(&tmY, slab, n0, wrow);
+                        bulk_commit_group();
+                    }
+                    last_group[buf] = committed++;
+                }
+                buf ^= 1;
+            }
+            ++acc_it;
+        }
+        if (lane == 0) bulk_wait_group_all();
+        __syncwarp();
+    }
+
+    // ---------------------------------------------------------------- teardown
+    __syncwarp();
+    if (warp == 1 && lane == 0 && rank == 0) {
+        tc_commit_pair(fin, 0x1);    // completes once every MMA of the pair is done
+        drain_wait(fin, 0, args.wait_ns, args.status);
+        if constexpr (NVF4) drain_wait(cp_fin, 0, args.wait_ns, args.status);
+    }
+    tc_fence_before();
+    cluster_sync();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tbase, kTmemCols);
+}
+
 // ---------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
@@ -365,20 +743,112 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// 2-D tensor [rows][inner] of `dtype`, box of box_rows x box_inner elements.
+int make_map_2d(CUtensorMap* m, CUtensorMapDataType dtype, uint32_t elem_bytes, const void* base,
+                uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows,
+                CUtensorMapSwizzle swizzle)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return BSP_ERR_CUDA;
+    cuuint64_t dims[2] = {inner, rows};
+    cuuint64_t strides[1] = {inner * elem_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_CUDA;
+}
+
 // 2-D byte tensor [rows][row_bytes], box of box_rows x 128 bytes, 128-byte swizzle.
 int make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
              uint32_t box_rows)
 {
-    EncodeTiledFn fn = encode_fn();
-    if (!fn) return BSP_ERR_CUDA;
-    cuuint64_t dims[2] = {row_bytes, rows};
-    cuuint64_t strides[1] = {row_bytes};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(kBKB), box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
-                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_CUDA;
+    return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, row_bytes, rows, kBKB, box_rows,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <bool NVF4>
+int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, int sms,
+                cudaStream_t s)
+{
+    using C = PairCfg<NVF4>;
+    static std::once_flag once[64];
+    static cudaError_t err[64];
+    static int max_pairs[64];
+    std::call_once(once[dev], [&] {
+        err[dev] = cudaFuncSetAttribute(gemm_pair_kernel<NVF4>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        max_pairs[dev] = sms / 2;
+        if (err[dev] == cudaSuccess) {
+            cudaLaunchConfig_t cfg = {};
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.gridDim = dim3(static_cast<unsigned>(sms), 1, 1);
+            cfg.blockDim = dim3(C::THREADS, 1, 1);
+            cfg.dynamicSmemBytes = C::SMEM_BYTES;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<NVF4>, &cfg) ==
+                    cudaSuccess &&
+                clusters > 0)
+                max_pairs[dev] = clusters < sms / 2 ? clusters : sms / 2;
+            else
+                cudaGetLastError();
+        }
+    });
+    if (err[dev] != cudaSuccess) return BSP_ERR_CUDA;
+    const uint64_t row_bytes = NVF4 ? static_cast<uint64_t>(args.K) / 2 : args.K;
+    CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
+    int st = make_map(&tmA, a, row_bytes, static_cast<uint64_t>(args.M), 128);
+    if (st == BSP_OK) st = make_map(&tmB, w, row_bytes, static_cast<uint64_t>(args.N), 128);
+    if (st == BSP_OK)
+        st = make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, args.out,
+                         static_cast<uint64_t>(args.N), static_cast<uint64_t>(args.M), 32, 32,
+                         CU_TENSOR_MAP_SWIZZLE_64B);
+    if (st != BSP_OK) return st;
+    if (NVF4) {
+        // scale arrays viewed as rows of 16 bytes; a box is 4 chunks of 512 bytes
+        const uint64_t sfa_rows = static_cast<uint64_t>(nvfp4_sf_bytes(args.M, args.K, BSP_SF_MMA)) / 16;
+        const uint64_t sfb_rows = static_cast<uint64_t>(nvfp4_sf_bytes(args.N, args.K, BSP_SF_MMA)) / 16;
+        st = make_map_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, args.sfa, 16, sfa_rows, 16, 128,
+                         CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st == BSP_OK)
+            st = make_map_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, args.sfb, 16, sfb_rows, 16,
+                             128, CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (st != BSP_OK) return st;
+    } else {
+        tmSFA = tmA;
+        tmSFB = tmA;
+    }
+    const int64_t tiles =
+        static_cast<int64_t>((args.M + 255) / 256) * ((args.N + 255) / 256);
+    const int pairs = static_cast<int>(tiles < max_pairs[dev] ? tiles : max_pairs[dev]);
+    gemm_pair_kernel<NVF4><<<2 * pairs, C::THREADS, C::SMEM_BYTES, s>>>(tmA, tmB, tmSFA, tmSFB,
+                                                                        tmY, args);
+    return launch_status();
+}
+
+// Kernel choice: 0 = automatic (CTA pairs with 256x256 tiles unless M fits one
+// 128-row tile), 1 = CTA pairs, 2 = single CTAs.  Initialised from the
+// BSP_GEMM_KERNEL environment variable ("pair" / "single"); tests can set it.
+std::atomic<int> g_kernel_choice{-1};
+
+int kernel_choice()
+{
+    int c = g_kernel_choice.load();
+    if (c < 0) {
+        const char* e = std::getenv("BSP_GEMM_KERNEL");
+        c = (e && std::strcmp(e, "pair") == 0) ? 1 : (e && std::strcmp(e, "single") == 0) ? 2 : 0;
+        int expected = -1;
+        g_kernel_choice.compare_exchange_strong(expected, c);
+        c = g_kernel_choice.load();
+    }
+    return c;
 }
 
 template <bool NVF4, int BN, int STAGES, int NACC>
@@ -457,6 +927,10 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     args.wait_ns = wait_ns_override ? wait_ns_override : wait_limit_ns();
     args.debug_stop_iter = debug_stop_iter;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int choice = kernel_choice();
+    const bool pair = choice == 1 || (choice == 0 && M > kBM);
+    if (pair) return nvf4 ? launch_pair<true>(a, w, args, dev, sms, s)
+                          : launch_pair<false>(a, w, args, dev, sms, s);
     if (nvf4) {
         if (N > 128) return launch<true, 256, 4, 1>(a, w, args, dev, sms, s);
         return launch<true, 128, 6, 2>(a, w, args, dev, sms, s);
@@ -485,6 +959,14 @@ int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_
 {
     return bsp::gemm_entry(false, a_e4m3, nullptr, a_row_scale, w_e4m3, nullptr, w_row_scale,
                            bias_bf16, out_bf16, M, N, K, stream, -1, 0);
+}
+
+int bsp_testing_set_gemm_kernel(int choice)
+{
+    if (choice < 0 || choice > 2) return BSP_ERR_INVALID_ARG;
+    const int old = bsp::kernel_choice();
+    bsp::g_kernel_choice.store(choice);
+    return old;
 }
 
 int bsp_testing_gemm_stall(int scheme, const uint8_t* a, const uint8_t* a_sf, const float* a_scale,

@@ -31,6 +31,15 @@ int bsp_testing_gemm_stall(int scheme, const uint8_t* a, const uint8_t* a_sf,
                            int64_t K, int64_t stop_after_stages, int64_t wait_limit_ms,
                            bsp_stream_t stream);
 
+/*
+ * bsp_testing_set_gemm_kernel -- selects the GEMM kernel of later nvfp4_gemm /
+ * fp8r_gemm calls in this process: 0 = automatic (default), 1 = CTA-pair kernel
+ * (256 x 256 tiles, tcgen05 cta_group::2), 2 = single-CTA kernel (128 x 256 or
+ * 128 x 128 tiles).  Both compute the same results; this exists so the tests can
+ * cover each.  Returns the previous choice, or BSP_ERR_INVALID_ARG.
+ */
+int bsp_testing_set_gemm_kernel(int choice);
+
 #ifdef __cplusplus
 }
 #endif

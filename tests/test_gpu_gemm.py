@@ -21,6 +21,15 @@ pytestmark = pytest.mark.gpu
 E2M1 = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 
 
+@pytest.fixture(params=["pair", "single"], autouse=True)
+def gemm_kernel(request):
+    """Run every GEMM test on both kernels: CTA pairs (256x256 tiles, cta_group::2)
+    and single CTAs (128-row tiles)."""
+    old = bsp.bsp_testing_set_gemm_kernel({"pair": 1, "single": 2}[request.param])
+    yield request.param
+    bsp.bsp_testing_set_gemm_kernel(old)
+
+
 # ------------------------------------------------------------------ NVFP4 path
 def gpu_nvfp4_linear(a_cpu, w_cpu, bias_cpu=None):
     """Whole CUDA path: device global scales, both quantizers, the GEMM."""
