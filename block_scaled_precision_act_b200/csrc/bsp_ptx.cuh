@@ -306,6 +306,28 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr)
                  : "memory");
 }
 
+// Relaxed arrive (no memory ordering) on an mbarrier given by its shared::cluster
+// address.  Much cheaper than the release form across CTAs; use it where the waiter
+// needs no data written by this thread (e.g. "the MMAs reading your stage are done").
+__device__ __forceinline__ void mbar_arrive_cluster_relaxed(uint32_t cluster_addr)
+{
+    asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(
+                     cluster_addr)
+                 : "memory");
+}
+
+// 3-D tensor load issued by either CTA of a pair, completing on the leader's barrier.
+__device__ __forceinline__ void tma_load_3d_pair(void* dst, const CUtensorMap* m,
+                                                 uint32_t bar_cluster_addr, int32_t x, int32_t y,
+                                                 int32_t z)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(bar_cluster_addr), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
+
 // 2-D tensor load issued by either CTA of a pair; the transaction bytes complete on
 // the mbarrier at `bar_cluster_addr` (the pair leader's barrier).  No multicast.
 __device__ __forceinline__ void tma_load_2d_pair(void* dst, const CUtensorMap* m,

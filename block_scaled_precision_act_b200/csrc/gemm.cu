@@ -485,19 +485,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         ok = false;
                         break;
                     }
+                    // The MMAs release a stage on CTA 0's barrier only; CTA 0 relays it to
+                    // CTA 1 with a relaxed arrive (a release-ordered cross-CTA arrive per
+                    // stage costs about half the load bandwidth).
+                    if (rank == 0 && it >= STAGES)
+                        mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(empty + s), 1));
                     const uint32_t bar0 = mapa_shared(smem_u32(full + s), 0);
                     if (rank == 0) mbar_arrive_expect_tx(full + s, 2 * C::STAGE_TX);
                     tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar0, kt * kBKB, a_row);
                     tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar0, kt * kBKB, b_row);
                     if constexpr (NVF4) {
-                        // scale chunks are 32 rows of 16 bytes; a stage needs 4 chunks
-                        const int ya = ((a_row / 128) * kb4 + 4 * kt) * 32;
-                        tma_load_2d_pair(sSFA + s * C::SFA_BYTES, &tmSFA, bar0, 0, ya);
-                        for (int c = 0; c < 2; ++c) {
-                            const int yb = ((nt * 2 + c) * kb4 + 4 * kt) * 32;
-                            tma_load_2d_pair(sSFB + s * C::SFB_BYTES + c * 2048, &tmSFB, bar0, 0,
-                                             yb);
-                        }
+                        // scale arrays as [row tile][512-byte chunk][64 x 8 bytes]: a stage
+                        // needs chunks 4kt..4kt+3 of one (A) or two (B) row tiles: one box each
+                        tma_load_3d_pair(sSFA + s * C::SFA_BYTES, &tmSFA, bar0, 0, 4 * kt,
+                                         a_row / 128);
+                        tma_load_3d_pair(sSFB + s * C::SFB_BYTES, &tmSFB, bar0, 0, 4 * kt, nt * 2);
                     }
                     ++it;
                 }
@@ -552,7 +554,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         else
                             mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::IDESC, acc);
                     }
-                    tc_commit_pair(empty + s, 0x3);
+                    tc_commit_pair(empty + s, 0x1);
                     if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
                     ++it;
                 }
@@ -637,9 +639,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 tmem_ld_wait();
                 // the shared subtiles are ord 0, 1, 2: half 0 holds two, half 1 one
                 if ((h == 0 && idx == 1) || (h == 1 && idx == 0)) {
+                    // values are in registers (wait::ld done): a relaxed arrive suffices
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(acc_empty0);
+                    if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty0);
                 }
                 const int n0 = nt * 256 + j * 32;
                 uint32_t packed[16];
@@ -760,6 +763,23 @@ int make_map_2d(CUtensorMap* m, CUtensorMapDataType dtype, uint32_t elem_bytes, 
     return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_CUDA;
 }
 
+// Block scales in the MMA layout as a 3-D tensor of 8-byte elements:
+// [row tiles][kb4 chunks of 512 bytes][64]; a box is 4 chunks of `tiles` row tiles.
+int make_map_sf(CUtensorMap* m, const void* base, uint64_t kb4, uint64_t row_tiles,
+                uint32_t tiles)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return BSP_ERR_CUDA;
+    cuuint64_t dims[3] = {64, kb4, row_tiles};
+    cuuint64_t strides[2] = {512, kb4 * 512};
+    cuuint32_t box[3] = {64, 4, tiles};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT64, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_CUDA;
+}
+
 // 2-D byte tensor [rows][row_bytes], box of box_rows x 128 bytes, 128-byte swizzle.
 int make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
              uint32_t box_rows)
@@ -812,14 +832,11 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
                          CU_TENSOR_MAP_SWIZZLE_64B);
     if (st != BSP_OK) return st;
     if (NVF4) {
-        // scale arrays viewed as rows of 16 bytes; a box is 4 chunks of 512 bytes
-        const uint64_t sfa_rows = static_cast<uint64_t>(nvfp4_sf_bytes(args.M, args.K, BSP_SF_MMA)) / 16;
-        const uint64_t sfb_rows = static_cast<uint64_t>(nvfp4_sf_bytes(args.N, args.K, BSP_SF_MMA)) / 16;
-        st = make_map_2d(&tmSFA, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, args.sfa, 16, sfa_rows, 16, 128,
-                         CU_TENSOR_MAP_SWIZZLE_NONE);
+        // scale arrays as [row tile][chunk][64 x 8 bytes]; boxes of 4 chunks x 1 or 2 tiles
+        const uint64_t kb4 = static_cast<uint64_t>(args.K / 16 + 3) / 4;
+        st = make_map_sf(&tmSFA, args.sfa, kb4, static_cast<uint64_t>(args.M + 127) / 128, 1);
         if (st == BSP_OK)
-            st = make_map_2d(&tmSFB, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, args.sfb, 16, sfb_rows, 16,
-                             128, CU_TENSOR_MAP_SWIZZLE_NONE);
+            st = make_map_sf(&tmSFB, args.sfb, kb4, static_cast<uint64_t>(args.N + 127) / 128, 2);
         if (st != BSP_OK) return st;
     } else {
         tmSFA = tmA;

@@ -23,7 +23,6 @@ namespace bsp {
 namespace {
 
 constexpr int kQuantThreads = 256;
-constexpr int kQuantUnroll = 4;
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p)
 {
@@ -48,12 +47,91 @@ __device__ __forceinline__ int64_t sf_mma_offset(int64_t row, int64_t kb, int64_
            (kb & 3);
 }
 
-// One warp-iteration handles 32*U consecutive "octets" (8 bf16 each); lanes 2j and
-// 2j+1 of an iteration hold the two halves of one 16-element block.
+// Each thread owns whole 16-element blocks (two 16-byte loads), two blocks per
+// iteration (block indices i and i + 32 within a 64-block warp span), with the next
+// iteration's loads issued before the current blocks are encoded.  Lanes 4j..4j+3 of
+// a warp hold 4 consecutive blocks of one row (K % 64 == 0 for the MMA layout), so the
+// 4 scale bytes are gathered by shuffles and written as one word.
+constexpr int kQBlocksPerWarp = 64;
+
+struct Block16 {
+    uint4 lo, hi;
+};
+
+__device__ __forceinline__ Block16 load_block(const uint4* x, int64_t blk, int64_t nblk)
+{
+    Block16 b;
+    if (blk < nblk) {
+        b.lo = ld_stream(x + 2 * blk);
+        b.hi = ld_stream(x + 2 * blk + 1);
+    } else {
+        b.lo = make_uint4(0, 0, 0, 0);
+        b.hi = b.lo;
+    }
+    return b;
+}
+
+// Encode one block: returns the 8 code bytes (element 2j in the low nibble) and the
+// E4M3 scale byte.
+__device__ __forceinline__ uint2 encode_block(const Block16& b, float g, float t, uint32_t& sb)
+{
+    float f[16];
+    unpack8(b.lo, *reinterpret_cast<float(*)[8]>(&f[0]));
+    unpack8(b.hi, *reinterpret_cast<float(*)[8]>(&f[8]));
+    float amax = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    const float s = (t > 0.0f) ? __fdiv_rn(amax, t) : 0.0f;
+    sb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
+    const float d = __fmul_rn(e4m3_to_f32(sb), g);
+    uint2 w = make_uint2(0, 0);
+    if (d != 0.0f) {
+        const float r = fminf(__frcp_rn(d), FLT_MAX);
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[i], r);
+        w.x = cvt_e2m1x8(y);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[8 + i], r);
+        w.y = cvt_e2m1x8(y);
+    }
+    return w;
+}
+
+template <int LAYOUT>
+__device__ __forceinline__ void store_block(uint2* codes, uint8_t* scales, int64_t blk,
+                                            int64_t nblk, int64_t nb_row, int64_t kb4, uint2 w,
+                                            uint32_t sb, int lane)
+{
+    // gather 4 consecutive blocks' scale bytes into lane 4j
+    const uint32_t s1 = __shfl_down_sync(0xffffffffu, sb, 1);
+    const uint32_t s2 = __shfl_down_sync(0xffffffffu, sb, 2);
+    const uint32_t s3 = __shfl_down_sync(0xffffffffu, sb, 3);
+    if (blk < nblk) {
+        codes[blk] = w;
+        if ((lane & 3) == 0) {
+            const uint32_t w4 = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
+            int64_t off;
+            if (LAYOUT == BSP_SF_LINEAR) {
+                off = blk;                                   // [rows][K/16] is the block index
+            } else {
+                const int64_t row = blk / nb_row;
+                off = sf_mma_offset(row, blk - row * nb_row, kb4);
+            }
+            if (blk + 3 < nblk && (off & 3) == 0) {
+                *reinterpret_cast<uint32_t*>(scales + off) = w4;
+            } else {                                         // ragged tail of a linear layout
+                for (int i = 0; i < 4 && blk + i < nblk; ++i)
+                    scales[off + i] = static_cast<uint8_t>(w4 >> (8 * i));
+            }
+        }
+    }
+}
+
 template <int LAYOUT>
 __global__ void __launch_bounds__(kQuantThreads)
-    nvfp4_quant_kernel(const uint4* __restrict__ x, int64_t total_oct, int64_t oct_per_row,
-                       const float* __restrict__ gptr, uint32_t* __restrict__ codes,
+    nvfp4_quant_kernel(const uint4* __restrict__ x, int64_t nblk, int64_t nb_row,
+                       const float* __restrict__ gptr, uint2* __restrict__ codes,
                        uint8_t* __restrict__ scales)
 {
     const float g = __ldg(gptr);
@@ -61,58 +139,25 @@ __global__ void __launch_bounds__(kQuantThreads)
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kQuantThreads) >> 5;
-    const int64_t nb_row = oct_per_row >> 1;        // blocks per row = K/16
-    const int64_t kb4 = (nb_row + 3) >> 2;          // MMA column tiles
+    const int64_t kb4 = (nb_row + 3) >> 2;
+    const int64_t step = nwarps * kQBlocksPerWarp;
 
-    for (int64_t base = warp * 32 * kQuantUnroll; base < total_oct;
-         base += nwarps * 32 * kQuantUnroll) {
-        uint4 v[kQuantUnroll];
-#pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t o = base + u * 32 + lane;
-            v[u] = (o < total_oct) ? ld_stream(x + o) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < kQuantUnroll; ++u) {
-            const int64_t o = base + u * 32 + lane;
-            float f[8];
-            unpack8(v[u], f);
-            float amax = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, 1));
-            const float s = (t > 0.0f) ? __fdiv_rn(amax, t) : 0.0f;
-            const uint32_t sb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
-            const float d = __fmul_rn(e4m3_to_f32(sb), g);
-            uint32_t word = 0;
-            if (d != 0.0f) {
-                const float r = fminf(__frcp_rn(d), FLT_MAX);
-                float y[8];
-#pragma unroll
-                for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[i], r);
-                word = cvt_e2m1x8(y);
-            }
-            if (LAYOUT == BSP_SF_LINEAR) {
-                if (o < total_oct) {
-                    codes[o] = word;
-                    if ((lane & 1) == 0) scales[o >> 1] = static_cast<uint8_t>(sb);
-                }
-            } else {
-                // gather the 4 scales of blocks kb..kb+3 (kb % 4 == 0) into lane 8i
-                const uint32_t s1 = __shfl_down_sync(0xffffffffu, sb, 2);
-                const uint32_t s2 = __shfl_down_sync(0xffffffffu, sb, 4);
-                const uint32_t s3 = __shfl_down_sync(0xffffffffu, sb, 6);
-                if (o < total_oct) {
-                    codes[o] = word;
-                    if ((lane & 7) == 0) {
-                        const int64_t row = o / oct_per_row;
-                        const int64_t kb = (o - row * oct_per_row) >> 1;
-                        const uint32_t w4 = sb | (s1 << 8) | (s2 << 16) | (s3 << 24);
-                        *reinterpret_cast<uint32_t*>(scales + sf_mma_offset(row, kb, kb4)) = w4;
-                    }
-                }
-            }
-        }
+    int64_t base = warp * kQBlocksPerWarp;
+    Block16 b0 = load_block(x, base + lane, nblk);
+    Block16 b1 = load_block(x, base + 32 + lane, nblk);
+    while (base < nblk) {
+        const int64_t next = base + step;
+        // prefetch the next span before encoding this one
+        Block16 n0 = load_block(x, next + lane, nblk);
+        Block16 n1 = load_block(x, next + 32 + lane, nblk);
+        uint32_t sb0, sb1;
+        const uint2 w0 = encode_block(b0, g, t, sb0);
+        store_block<LAYOUT>(codes, scales, base + lane, nblk, nb_row, kb4, w0, sb0, lane);
+        const uint2 w1 = encode_block(b1, g, t, sb1);
+        store_block<LAYOUT>(codes, scales, base + 32 + lane, nblk, nb_row, kb4, w1, sb1, lane);
+        b0 = n0;
+        b1 = n1;
+        base = next;
     }
 }
 
@@ -286,17 +331,18 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
     int dev = 0, sms = 0;
     int st = check_device(&dev, &sms);
     if (st != BSP_OK) return st;
-    const int64_t total_oct = M * (K / 8);
-    const int grid = grid_for(total_oct, kQuantThreads * kQuantUnroll, sms, 8);
+    const int64_t nblk = M * (K / 16);
+    // at most the resident grid (4 CTAs of 256 threads per SM at 64 registers)
+    const int grid = grid_for(nblk, (kQuantThreads / 32) * kQBlocksPerWarp, sms, 4);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (layout == BSP_SF_LINEAR)
         nvfp4_quant_kernel<BSP_SF_LINEAR><<<grid, kQuantThreads, 0, s>>>(
-            static_cast<const uint4*>(x_bf16), total_oct, K / 8, global_scale,
-            reinterpret_cast<uint32_t*>(codes), scales);
+            static_cast<const uint4*>(x_bf16), nblk, K / 16, global_scale,
+            reinterpret_cast<uint2*>(codes), scales);
     else
         nvfp4_quant_kernel<BSP_SF_MMA><<<grid, kQuantThreads, 0, s>>>(
-            static_cast<const uint4*>(x_bf16), total_oct, K / 8, global_scale,
-            reinterpret_cast<uint32_t*>(codes), scales);
+            static_cast<const uint4*>(x_bf16), nblk, K / 16, global_scale,
+            reinterpret_cast<uint2*>(codes), scales);
     return launch_status();
 }
 
