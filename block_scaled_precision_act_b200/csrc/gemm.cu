@@ -615,6 +615,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         int buf = 0;
         int committed = 0;               // bulk-store groups this warp committed
         int last_group[2] = {-1, -1};    // group that last read each slab
+        const uint64_t out_policy = l2_policy_evict_first();
         for (int tile = pair; tile < num_tiles; tile += npairs) {
             const int mt = tile % num_m, nt = tile / num_m;
             const bool ok = mbar_wait(acc_full, static_cast<uint32_t>(acc_it & 1), abort_flag,
@@ -628,23 +629,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             if constexpr (!NVF4) sa = (m < M) ? __ldg(args.a_scale + m) : 0.0f;
             const uint32_t tq = tbase + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(sacc * C::ACC_STRIDE);
-            // subtiles of 32 columns; the 3 shared with the other accumulator come first
-            // (columns 160..255 of accumulator 0, columns 0..95 of accumulator 1)
-#pragma unroll 1
+            // Subtiles of 32 columns.  The 3 shared with the other accumulator (columns
+            // 160..255 of accumulator 0, 0..95 of accumulator 1) come first: this warp's
+            // share of them (two for half 0, one for half 1) is read from TMEM before
+            // anything else, then the accumulator is released to the MMA thread.
+            uint32_t pre[2][32];
+            const int npre = (h == 0) ? 2 : 1;
+#pragma unroll
+            for (int idx = 0; idx < 2; ++idx) {
+                if (idx < npre) {
+                    const int ord = 2 * idx + h;
+                    const int j = sacc == 0 ? (ord + 5) & 7 : ord;
+                    tmem_ld_x32(tq + j * 32, pre[idx]);
+                }
+            }
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty0);   // values are in registers
+#pragma unroll
             for (int idx = 0; idx < 4; ++idx) {
                 const int ord = 2 * idx + h;                        // 0..7
                 const int j = sacc == 0 ? (ord + 5) & 7 : ord;
-                uint32_t r[32];
-                tmem_ld_x32(tq + j * 32, r);
-                tmem_ld_wait();
-                // the shared subtiles are ord 0, 1, 2: half 0 holds two, half 1 one
-                if ((h == 0 && idx == 1) || (h == 1 && idx == 0)) {
-                    // values are in registers (wait::ld done): a relaxed arrive suffices
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty0);
-                }
                 const int n0 = nt * 256 + j * 32;
+                uint32_t r[32];
+                if (idx < npre) {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) r[i] = (idx == 0) ? pre[0][i] : pre[1][i];
+                } else {
+                    tmem_ld_x32(tq + j * 32, r);
+                    tmem_ld_wait();
+                }
                 uint32_t packed[16];
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
@@ -697,7 +712,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 __syncwarp();
                 if (wrow < M && n0 < N) {
                     if (lane == 0) {
-                        tma_store_2d(&tmY, slab, n0, wrow);
+                        tma_store_2d_hint(&tmY, slab, n0, wrow, out_policy);
                         bulk_commit_group();
                     }
                     last_group[buf] = committed++;
