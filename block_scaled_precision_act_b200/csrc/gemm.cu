@@ -368,13 +368,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 // a TMA store.
 template <bool NVF4>
 struct PairCfg {
-    static constexpr int STAGES = NVF4 ? 5 : 6;
+    // A stage holds ATOMS K-atoms (128 rows x 128 bytes each) of A and of B.  NVFP4 keeps
+    // one-atom stages so its scale copies pipeline per atom; FP8 takes two-atom stages
+    // (half the TMA instructions and barrier round trips per byte).
+    static constexpr int ATOMS = NVF4 ? 1 : 2;
+    static constexpr int STAGES = NVF4 ? 5 : 3;
     static constexpr int THREADS = 13 * 32;
-    static constexpr int A_BYTES = 128 * kBKB;
-    static constexpr int B_BYTES = 128 * kBKB;
+    static constexpr int ATOM = 128 * kBKB;
+    static constexpr int A_BYTES = ATOMS * ATOM;
+    static constexpr int B_BYTES = ATOMS * ATOM;
     static constexpr int SFA_BYTES = NVF4 ? 2048 : 0;
     static constexpr int SFB_BYTES = NVF4 ? 4096 : 0;
-    static constexpr int K_STAGE = NVF4 ? 256 : 128;
+    static constexpr int K_STAGE = NVF4 ? 256 : 128 * ATOMS;
     static constexpr int K_MMA = NVF4 ? 64 : 32;
     static constexpr int STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;
     static constexpr int EPI_WARPS = 8;
@@ -393,6 +398,7 @@ struct PairCfg {
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(OFF_EPI % 1024 == 0, "epilogue slabs must be 1024-byte aligned");
     static_assert(SF_COL0 + 2 * SF_BUF <= 512 && ACC_STRIDE + 256 <= SF_COL0, "TMEM budget");
+    static_assert(!NVF4 || ATOMS == 1, "scale copies are staged per atom");
 };
 
 template <bool NVF4>
@@ -492,8 +498,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(empty + s), 1));
                     const uint32_t bar0 = mapa_shared(smem_u32(full + s), 0);
                     if (rank == 0) mbar_arrive_expect_tx(full + s, 2 * C::STAGE_TX);
-                    tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar0, kt * kBKB, a_row);
-                    tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar0, kt * kBKB, b_row);
+                    if constexpr (C::ATOMS == 1) {
+                        tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar0, kt * kBKB, a_row);
+                        tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar0, kt * kBKB, b_row);
+                    } else {
+                        // operands viewed as [atom][row][128 B]: one box = 128 rows x ATOMS atoms
+                        tma_load_3d_pair(sA + s * C::A_BYTES, &tmA, bar0, 0, a_row, C::ATOMS * kt);
+                        tma_load_3d_pair(sB + s * C::B_BYTES, &tmB, bar0, 0, b_row, C::ATOMS * kt);
+                    }
                     if constexpr (NVF4) {
                         // scale arrays as [row tile][512-byte chunk][64 x 8 bytes]: a stage
                         // needs chunks 4kt..4kt+3 of one (A) or two (B) row tiles: one box each
@@ -541,18 +553,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         tc_fence_after();
                         nk = min(4, K / 64 - 4 * kt);
                     } else {
-                        nk = min(4, (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
+                        nk = min(4 * C::ATOMS, (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
                     }
                     const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + s * C::A_BYTES));
                     const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * C::B_BYTES));
                     const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
                     for (int k = 0; k < nk; ++k) {
                         const uint32_t acc = (kt > 0 || k > 0) ? 1u : 0u;
+                        // K-step k lies in atom k/4 (ATOM bytes further on: ATOM/16 in the
+                        // descriptor's address field), 32 bytes (2) per step inside it
+                        const uint64_t koff = static_cast<uint64_t>((k >> 2) * (C::ATOM >> 4) +
+                                                                    2 * (k & 3));
                         if constexpr (NVF4)
-                            mma_nvf4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::IDESC, sf + k * 4,
+                            mma_nvf4_pair(d_tmem, adesc + koff, bdesc + koff, C::IDESC, sf + k * 4,
                                           sf + 16 + k * 8, acc);
                         else
-                            mma_f8f6f4_pair(d_tmem, adesc + 2 * k, bdesc + 2 * k, C::IDESC, acc);
+                            mma_f8f6f4_pair(d_tmem, adesc + koff, bdesc + koff, C::IDESC, acc);
                     }
                     tc_commit_pair(empty + s, 0x1);
                     if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
@@ -795,6 +811,25 @@ int make_map_sf(CUtensorMap* m, const void* base, uint64_t kb4, uint64_t row_til
     return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_CUDA;
 }
 
+// Operand codes [rows][row_bytes] viewed as [row_bytes/128 atoms][rows][128 B] (the atom
+// dimension has the smaller stride); a box is 128 rows x `atoms` atoms, 128-byte swizzle,
+// so one TMA instruction brings atoms x 128 bytes of K for 128 rows.  Needs
+// row_bytes % 128 == 0.
+int make_map_atoms(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
+                   uint32_t atoms)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return BSP_ERR_CUDA;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(kBKB), rows, row_bytes / kBKB};
+    cuuint64_t strides[2] = {row_bytes, static_cast<cuuint64_t>(kBKB)};
+    cuuint32_t box[3] = {static_cast<cuuint32_t>(kBKB), 128, atoms};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? BSP_OK : BSP_ERR_CUDA;
+}
+
 // 2-D byte tensor [rows][row_bytes], box of box_rows x 128 bytes, 128-byte swizzle.
 int make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows,
              uint32_t box_rows)
@@ -839,8 +874,16 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
     if (err[dev] != cudaSuccess) return BSP_ERR_CUDA;
     const uint64_t row_bytes = NVF4 ? static_cast<uint64_t>(args.K) / 2 : args.K;
     CUtensorMap tmA, tmB, tmSFA, tmSFB, tmY;
-    int st = make_map(&tmA, a, row_bytes, static_cast<uint64_t>(args.M), 128);
-    if (st == BSP_OK) st = make_map(&tmB, w, row_bytes, static_cast<uint64_t>(args.N), 128);
+    int st;
+    if (C::ATOMS == 1) {
+        st = make_map(&tmA, a, row_bytes, static_cast<uint64_t>(args.M), 128);
+        if (st == BSP_OK) st = make_map(&tmB, w, row_bytes, static_cast<uint64_t>(args.N), 128);
+    } else {
+        if (row_bytes % kBKB != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
+        st = make_map_atoms(&tmA, a, row_bytes, static_cast<uint64_t>(args.M), C::ATOMS);
+        if (st == BSP_OK)
+            st = make_map_atoms(&tmB, w, row_bytes, static_cast<uint64_t>(args.N), C::ATOMS);
+    }
     if (st == BSP_OK)
         st = make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, args.out,
                          static_cast<uint64_t>(args.N), static_cast<uint64_t>(args.M), 32, 32,
@@ -960,7 +1003,9 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     args.debug_stop_iter = debug_stop_iter;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int choice = kernel_choice();
-    const bool pair = choice == 1 || (choice == 0 && M > kBM);
+    // the FP8 pair kernel loads whole 128-byte K-atoms (3-D boxes): K % 128 == 0
+    const bool pair_ok = nvf4 || K % kBKB == 0;
+    const bool pair = pair_ok && (choice == 1 || (choice == 0 && M > kBM));
     if (pair) return nvf4 ? launch_pair<true>(a, w, args, dev, sms, s)
                           : launch_pair<false>(a, w, args, dev, sms, s);
     if (nvf4) {

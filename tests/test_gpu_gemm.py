@@ -73,6 +73,8 @@ def check_nvfp4(a_cpu, w_cpu, bias_cpu=None, step=1):
     (200, 136, 320, 3),      # ragged M, N, and K not a multiple of the 256-wide stage
     (1, 8, 64, 4),           # degenerate: one row, one 8-column group
     (130, 264, 1216, 5),     # ragged everything, 19 K-blocks of 64
+    (200, 136, 768, 6),      # 3 K-atoms of 128 bytes: the pair kernel's last stage is half empty
+    (384, 512, 1280, 7),     # 5 K-atoms, N two full tiles
 ])
 def test_nvfp4_linear_small(M, N, K, seed):
     a = synth.bf16_normal((M, K), 1.0, seed, 0.01, 20.0)
@@ -223,7 +225,7 @@ def check_fp8r(a_cpu, w_cpu, bias_cpu=None, step=1):
 
 @pytest.mark.parametrize("M,N,K,seed", [
     (128, 256, 256, 0), (128, 128, 32, 1), (200, 136, 336, 2), (1, 8, 16, 3),
-    (300, 520, 1040, 4),
+    (300, 520, 1040, 4), (300, 520, 384, 5), (260, 264, 640, 6),
 ])
 def test_fp8r_linear_small(M, N, K, seed):
     a = synth.bf16_normal((M, K), 1.0, seed, 0.01, 20.0)
