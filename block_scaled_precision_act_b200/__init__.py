@@ -21,6 +21,7 @@ import torch
 __all__ = [
     "BSPError", "SF_LINEAR", "SF_MMA", "lib", "library_path",
     "nvfp4_quantize_act", "nvfp4_gemm", "fp8r_quantize_rows", "fp8r_gemm",
+    "nvfp4_linear", "nvfp4_linear_workspace_bytes",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
     "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel",
@@ -40,6 +41,9 @@ _SIGS = {
     "nvfp4_quantize_act": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_int, _c_vp], _c_int),
     "nvfp4_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                     _c_i64, _c_vp], _c_int),
+    "nvfp4_linear": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64,
+                      _c_vp, _c_i64, _c_vp], _c_int),
+    "nvfp4_linear_workspace_bytes": ([_c_i64, _c_i64], _c_i64),
     "fp8r_quantize_rows": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp], _c_int),
     "fp8r_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp],
                   _c_int),
@@ -158,6 +162,36 @@ def nvfp4_gemm(a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias=None, out=
            lib().nvfp4_gemm(_ptr(a_codes), _ptr(a_sf), _ptr(a_global), _ptr(w_codes),
                             _ptr(w_sf), _ptr(w_global), _ptr(bias), _ptr(out), M, N, 2 * K2,
                             _stream(stream)))
+    return out
+
+
+def nvfp4_linear_workspace_bytes(M: int, K: int) -> int:
+    n = lib().nvfp4_linear_workspace_bytes(M, K)
+    if n < 0:
+        raise BSPError("nvfp4_linear_workspace_bytes", int(n))
+    return int(n)
+
+
+def nvfp4_linear(x: torch.Tensor, input_scale: torch.Tensor, w_codes, w_sf, w_scale, bias=None,
+                 out=None, workspace=None, stream=None):
+    """Y[M, N] bf16 = nvfp4 linear of bf16 x [M, K]: activation quantizer + FP4 GEMM in one
+    call (the GEMM overlaps the quantizer's tail).  `workspace` (uint8, at least
+    nvfp4_linear_workspace_bytes(M, K) bytes) is allocated here when not given."""
+    _dtype(x, torch.bfloat16, "x")
+    _dtype(input_scale, torch.float32, "input_scale")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K:
+        raise BSPError("nvfp4_linear (K mismatch)", -1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((max(nvfp4_linear_workspace_bytes(M, K), 0),), dtype=torch.uint8,
+                                device=x.device)
+    _check("nvfp4_linear",
+           lib().nvfp4_linear(_ptr(x), _ptr(input_scale), _ptr(w_codes), _ptr(w_sf),
+                              _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K, _ptr(workspace),
+                              workspace.numel(), _stream(stream)))
     return out
 
 

@@ -126,7 +126,7 @@ const char* bsp_status_string(int status)
     }
 }
 
-int bsp_version(void) { return 100; }
+int bsp_version(void) { return 200; }
 
 int64_t nvfp4_sf_bytes(int64_t rows, int64_t K, int layout)
 {

@@ -104,6 +104,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
+// ----------------------------------------------------------------- programmatic dependent launch
+// Block until every grid this one depends on (a launch with programmatic stream
+// serialisation) has completed and its memory writes are visible; a no-op for a
+// grid launched the ordinary way.
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// Let the next grid in the stream, if launched with programmatic stream
+// serialisation, start its prologue; its griddep_wait() still waits for this grid.
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------- TMA / bulk copies
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* m)
 {

@@ -28,6 +28,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <mutex>
+#include <utility>
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -152,6 +153,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
+            // Under a programmatic launch the operands may still be being written by
+            // the preceding grid (the activation quantizer): nothing is loaded before
+            // it has completed.  Everything else in the kernel follows these loads.
+            griddep_wait();
             int64_t it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
@@ -477,6 +482,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
+            // Under a programmatic launch the operands may still be being written by
+            // the preceding grid (the activation quantizer): nothing is loaded before
+            // it has completed.  Everything else in the kernel follows these loads.
+            griddep_wait();
             int64_t it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
@@ -838,9 +847,30 @@ int make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows
                        CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
+// Launch `kernel`; with `pdl` the launch allows programmatic stream serialisation, so
+// the grid may start (prologue: barriers, TMEM, tensor-map prefetch) while the
+// preceding grid in the stream finishes.  The kernels' producers call griddep_wait()
+// before their first load.
+template <typename... Params, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                          cudaStream_t s, bool pdl, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <bool NVF4>
 int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, int sms,
-                cudaStream_t s)
+                cudaStream_t s, bool pdl)
 {
     using C = PairCfg<NVF4>;
     static std::once_flag once[64];
@@ -903,8 +933,11 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
     const int64_t tiles =
         static_cast<int64_t>((args.M + 255) / 256) * ((args.N + 255) / 256);
     const int pairs = static_cast<int>(tiles < max_pairs[dev] ? tiles : max_pairs[dev]);
-    gemm_pair_kernel<NVF4><<<2 * pairs, C::THREADS, C::SMEM_BYTES, s>>>(tmA, tmB, tmSFA, tmSFB,
-                                                                        tmY, args);
+    if (launch_kernel(gemm_pair_kernel<NVF4>, 2 * pairs, C::THREADS, C::SMEM_BYTES, s, pdl, tmA,
+                      tmB, tmSFA, tmSFB, tmY, args) != cudaSuccess) {
+        cudaGetLastError();
+        return BSP_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -928,7 +961,7 @@ int kernel_choice()
 
 template <bool NVF4, int BN, int STAGES, int NACC>
 int launch(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, int sms,
-           cudaStream_t s)
+           cudaStream_t s, bool pdl)
 {
     using C = Cfg<NVF4, BN, STAGES, NACC>;
     static std::once_flag attr_once[64];
@@ -948,7 +981,11 @@ int launch(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, in
     const int64_t tiles =
         static_cast<int64_t>((args.M + kBM - 1) / kBM) * ((args.N + BN - 1) / BN);
     const int grid = static_cast<int>(tiles < sms ? tiles : sms);
-    gemm_kernel<NVF4, BN, STAGES, NACC><<<grid, kThreads, C::SMEM_BYTES, s>>>(tmA, tmB, args);
+    if (launch_kernel(gemm_kernel<NVF4, BN, STAGES, NACC>, grid, kThreads, C::SMEM_BYTES, s, pdl,
+                      tmA, tmB, args) != cudaSuccess) {
+        cudaGetLastError();
+        return BSP_ERR_CUDA;
+    }
     return launch_status();
 }
 
@@ -969,7 +1006,7 @@ int check_gemm_common(const void* a, const void* w, const void* bias, const void
 int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_scale,
                const uint8_t* w, const uint8_t* sfb, const float* w_scale, const void* bias,
                void* out, int64_t M, int64_t N, int64_t K, bsp_stream_t stream,
-               int64_t debug_stop_iter, uint64_t wait_ns_override)
+               int64_t debug_stop_iter, uint64_t wait_ns_override, bool pdl)
 {
     int st = check_gemm_common(a, w, bias, out, M, N, K);
     if (st != BSP_OK || M == 0 || N == 0) return st;
@@ -1006,17 +1043,27 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     // the FP8 pair kernel loads whole 128-byte K-atoms (3-D boxes): K % 128 == 0
     const bool pair_ok = nvf4 || K % kBKB == 0;
     const bool pair = pair_ok && (choice == 1 || (choice == 0 && M > kBM));
-    if (pair) return nvf4 ? launch_pair<true>(a, w, args, dev, sms, s)
-                          : launch_pair<false>(a, w, args, dev, sms, s);
+    if (pair) return nvf4 ? launch_pair<true>(a, w, args, dev, sms, s, pdl)
+                          : launch_pair<false>(a, w, args, dev, sms, s, pdl);
     if (nvf4) {
-        if (N > 128) return launch<true, 256, 4, 1>(a, w, args, dev, sms, s);
-        return launch<true, 128, 6, 2>(a, w, args, dev, sms, s);
+        if (N > 128) return launch<true, 256, 4, 1>(a, w, args, dev, sms, s, pdl);
+        return launch<true, 128, 6, 2>(a, w, args, dev, sms, s, pdl);
     }
-    if (N > 128) return launch<false, 256, 4, 2>(a, w, args, dev, sms, s);
-    return launch<false, 128, 6, 2>(a, w, args, dev, sms, s);
+    if (N > 128) return launch<false, 256, 4, 2>(a, w, args, dev, sms, s, pdl);
+    return launch<false, 128, 6, 2>(a, w, args, dev, sms, s, pdl);
 }
 
 }  // namespace
+
+int nvfp4_gemm_dependent(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                         const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                         const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
+                         bsp_stream_t stream)
+{
+    return gemm_entry(true, a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias_bf16,
+                      out_bf16, M, N, K, stream, -1, 0, true);
+}
+
 }  // namespace bsp
 
 extern "C" {
@@ -1027,7 +1074,7 @@ int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_globa
                bsp_stream_t stream)
 {
     return bsp::gemm_entry(true, a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias_bf16,
-                           out_bf16, M, N, K, stream, -1, 0);
+                           out_bf16, M, N, K, stream, -1, 0, false);
 }
 
 int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_e4m3,
@@ -1035,7 +1082,7 @@ int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_
               int64_t N, int64_t K, bsp_stream_t stream)
 {
     return bsp::gemm_entry(false, a_e4m3, nullptr, a_row_scale, w_e4m3, nullptr, w_row_scale,
-                           bias_bf16, out_bf16, M, N, K, stream, -1, 0);
+                           bias_bf16, out_bf16, M, N, K, stream, -1, 0, false);
 }
 
 int bsp_testing_set_gemm_kernel(int choice)
@@ -1056,7 +1103,7 @@ int bsp_testing_gemm_stall(int scheme, const uint8_t* a, const uint8_t* a_sf, co
     if (scheme != 0 && scheme != 1) return BSP_ERR_INVALID_ARG;
     return bsp::gemm_entry(scheme == 1, a, a_sf, a_scale, w, w_sf, w_scale, nullptr, out_bf16, M,
                            N, K, stream, stop_after_stages,
-                           static_cast<uint64_t>(wait_limit_ms) * 1000000ull);
+                           static_cast<uint64_t>(wait_limit_ms) * 1000000ull, false);
 }
 
 }  // extern "C"

@@ -134,6 +134,9 @@ __global__ void __launch_bounds__(kQuantThreads)
                        const float* __restrict__ gptr, uint2* __restrict__ codes,
                        uint8_t* __restrict__ scales)
 {
+    // a GEMM launched as this grid's programmatic dependent may start its prologue now;
+    // it still waits for this grid to complete before reading the codes
+    griddep_launch_dependents();
     const float g = __ldg(gptr);
     const float t = __fmul_rn(6.0f, g);
     const int lane = threadIdx.x & 31;

@@ -110,6 +110,38 @@ int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_globa
                bsp_stream_t stream);
 
 /*
+ * nvfp4_linear -- the nvfp4 linear forward in one call ("BFL (fp8r / nvfp4)", Kernels
+ * table: the activations are quantized at run time, then the fused FP4 GEMM runs):
+ * nvfp4_quantize_act(x, input_scale) into `workspace` (BSP_SF_MMA scales), then
+ * nvfp4_gemm against the pre-quantized weights.  The GEMM is launched with
+ * programmatic stream serialisation, so its prologue overlaps the end of the
+ * quantizer; it reads no input before the quantizer has completed.  Results are
+ * bit-identical to the two separate calls.
+ *
+ *   x_bf16        [M][K] bf16 activations.
+ *   input_scale   device pointer to one fp32: the activation global scale g.
+ *   w_codes, w_sf, w_scale   the quantized weight: [N][K/2] codes, BSP_SF_MMA scales
+ *                 (rows = N), device fp32 weight_scale_2.
+ *   bias_bf16     [N] bf16 or NULL.   out_bf16  [M][N] bf16.
+ *   workspace     caller-owned device buffer of at least
+ *                 nvfp4_linear_workspace_bytes(M, K) bytes, 16-byte aligned.  It receives
+ *                 the quantized activations (codes, then scales at a 256-byte boundary),
+ *                 is fully overwritten by every call, and must not be in use by another
+ *                 call that can run at the same time (another stream).
+ * Constraints: K % 64 == 0, K >= 64, N % 8 == 0 (those of the two calls).
+ * Errors: BSP_ERR_INVALID_ARG when workspace is NULL or workspace_bytes too small;
+ * otherwise as nvfp4_quantize_act and nvfp4_gemm.
+ */
+int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_codes,
+                 const uint8_t* w_sf, const float* w_scale, const void* bias_bf16,
+                 void* out_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                 int64_t workspace_bytes, bsp_stream_t stream);
+
+/* Workspace bytes nvfp4_linear needs for an [M][K] activation (codes, padding to 256
+ * bytes, MMA-layout scales); negative on bad arguments. */
+int64_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
  * fp8r_quantize_rows -- per-row E4M3 quantizer ("BFL (fp8r / nvfp4)", fp8r bullet:
  * activations are quantized to E4M3 per row at run time; weights use one fp32 scale
  * per row).

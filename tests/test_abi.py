@@ -100,6 +100,23 @@ def test_gemm_validation_on_host():
     assert c(P, P, 128, 48, 0, 1, None) == SHAPE
 
 
+def test_linear_workspace_and_validation_on_host():
+    L = bsp.lib()
+    for M, K in [(1, 64), (4096, 3072), (200, 320), (0, 128)]:
+        codes = M * K // 2
+        expect = (codes + 255) // 256 * 256 + oracle.sf_bytes(M, K, True)
+        assert bsp.nvfp4_linear_workspace_bytes(M, K) == expect
+    assert L.nvfp4_linear_workspace_bytes(128, 96) == INVALID
+    assert L.nvfp4_linear_workspace_bytes(-1, 64) == INVALID
+    lin = L.nvfp4_linear
+    need = bsp.nvfp4_linear_workspace_bytes(128, 256)
+    assert lin(P, P, P, P, P, None, P, 128, 128, 256, None, need, None) == INVALID
+    assert lin(P, P, P, P, P, None, P, 128, 128, 256, P, need - 1, None) == INVALID
+    assert lin(P, P, P, P, P, None, P, 128, 128, 96, P, need, None) == SHAPE
+    assert lin(P, P, P, P, P, None, P, 128, 128, 256, P + 8, need, None) == MISALIGNED
+    assert lin(P, P, P, P, P, None, P, 0, 128, 256, None, 0, None) == OK   # empty problem
+
+
 def test_testing_hook_validation():
     L = bsp.lib()
     h = L.bsp_testing_gemm_stall
