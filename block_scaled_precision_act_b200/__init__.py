@@ -21,7 +21,8 @@ import torch
 __all__ = [
     "BSPError", "SF_LINEAR", "SF_MMA", "lib", "library_path",
     "nvfp4_quantize_act", "nvfp4_gemm", "fp8r_quantize_rows", "fp8r_gemm",
-    "nvfp4_linear", "nvfp4_linear_workspace_bytes",
+    "nvfp4_linear", "nvfp4_linear_workspace_bytes", "nvfp4_linear_noalloc",
+    "nvfp4_linear_noalloc_max_bytes",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
     "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel",
@@ -44,6 +45,9 @@ _SIGS = {
     "nvfp4_linear": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64,
                       _c_vp, _c_i64, _c_vp], _c_int),
     "nvfp4_linear_workspace_bytes": ([_c_i64, _c_i64], _c_i64),
+    "nvfp4_linear_noalloc": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
+                              _c_i64, _c_vp], _c_int),
+    "nvfp4_linear_noalloc_max_bytes": ([], _c_i64),
     "fp8r_quantize_rows": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp], _c_int),
     "fp8r_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp],
                   _c_int),
@@ -192,6 +196,29 @@ def nvfp4_linear(x: torch.Tensor, input_scale: torch.Tensor, w_codes, w_sf, w_sc
            lib().nvfp4_linear(_ptr(x), _ptr(input_scale), _ptr(w_codes), _ptr(w_sf),
                               _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K, _ptr(workspace),
                               workspace.numel(), _stream(stream)))
+    return out
+
+
+def nvfp4_linear_noalloc_max_bytes() -> int:
+    return int(lib().nvfp4_linear_noalloc_max_bytes())
+
+
+def nvfp4_linear_noalloc(x: torch.Tensor, input_scale: torch.Tensor, w_codes, w_sf, w_scale,
+                         out: torch.Tensor, bias=None, stream=None):
+    """nvfp4_linear with the library's own per-device buffer as workspace; allocates
+    nothing, so `out` ([M, N] bf16) must be given.  Calls that can run concurrently on
+    one device race on that buffer (see include/bsp.h)."""
+    _dtype(x, torch.bfloat16, "x")
+    _dtype(input_scale, torch.float32, "input_scale")
+    _dtype(out, torch.bfloat16, "out")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K or tuple(out.shape) != (M, N):
+        raise BSPError("nvfp4_linear_noalloc (shape mismatch)", -1)
+    _check("nvfp4_linear_noalloc",
+           lib().nvfp4_linear_noalloc(_ptr(x), _ptr(input_scale), _ptr(w_codes), _ptr(w_sf),
+                                      _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K,
+                                      _stream(stream)))
     return out
 
 

@@ -16,7 +16,7 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libbsp.so")
-SOURCES = ["api_common.cu", "quant.cu", "gemm.cu", "linear.cu"]
+SOURCES = ["api_common.cu", "quant.cu", "gemm.cu", "linear.cu", "linear_noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 

@@ -142,6 +142,33 @@ int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_
 int64_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
 
 /*
+ * nvfp4_linear_noalloc -- nvfp4_linear without a caller workspace and without any
+ * allocation.  The pages have no counterpart: this is a deployment variant of
+ * nvfp4_linear for callers that must not allocate device memory after start-up (a
+ * serving loop with a fixed memory plan, C code without an allocator): cudaMalloc /
+ * cudaFree can synchronise the device and fail under memory pressure.
+ *
+ * Arguments and results: those of nvfp4_linear minus workspace / workspace_bytes;
+ * results are bit-identical to nvfp4_linear.  The quantized activations go to one
+ * buffer of nvfp4_linear_noalloc_max_bytes() bytes (128 MiB) per device, compiled
+ * into the library (a file-scope __device__ array); its address is looked up on the
+ * first call on each device, so make that first call outside any stream capture.
+ * Nothing in it needs to start at zero (each call writes what it reads).
+ * Errors: BSP_ERR_UNSUPPORTED_SHAPE when nvfp4_linear_workspace_bytes(M, K) exceeds
+ * the buffer; otherwise as nvfp4_linear.
+ * Concurrency: the buffer is shared by all calls on a device, so calls that can run
+ * at the same time (different streams, unordered host threads) race on it and
+ * corrupt each other's results; calls ordered on one stream are safe.
+ */
+int nvfp4_linear_noalloc(const void* x_bf16, const float* input_scale, const uint8_t* w_codes,
+                         const uint8_t* w_sf, const float* w_scale, const void* bias_bf16,
+                         void* out_bf16, int64_t M, int64_t N, int64_t K, bsp_stream_t stream);
+
+/* Size in bytes of nvfp4_linear_noalloc's per-device buffer (the largest workspace it
+ * accepts). */
+int64_t nvfp4_linear_noalloc_max_bytes(void);
+
+/*
  * fp8r_quantize_rows -- per-row E4M3 quantizer ("BFL (fp8r / nvfp4)", fp8r bullet:
  * activations are quantized to E4M3 per row at run time; weights use one fp32 scale
  * per row).

@@ -117,6 +117,19 @@ def test_linear_workspace_and_validation_on_host():
     assert lin(P, P, P, P, P, None, P, 0, 128, 256, None, 0, None) == OK   # empty problem
 
 
+def test_noalloc_size_limit_on_host():
+    L = bsp.lib()
+    cap = bsp.nvfp4_linear_noalloc_max_bytes()
+    assert cap == 128 << 20
+    K = 3072
+    rows_ok = 4096
+    assert bsp.nvfp4_linear_workspace_bytes(rows_ok, K) <= cap
+    rows_big = cap // (K // 2) + 1
+    assert L.nvfp4_linear_noalloc(P, P, P, P, P, None, P, rows_big, 256, K, None) == SHAPE
+    assert L.nvfp4_linear_noalloc(P, P, P, P, P, None, P, 128, 128, 96, None) == SHAPE
+    assert L.nvfp4_linear_noalloc(P, P, P, P, P, None, P, 0, 128, 256, None) == OK
+
+
 def test_testing_hook_validation():
     L = bsp.lib()
     h = L.bsp_testing_gemm_stall
