@@ -71,16 +71,38 @@ __device__ __forceinline__ Block16 load_block(const uint4* x, int64_t blk, int64
     return b;
 }
 
+// max of two pairs of non-negative bf16 (NaN loses to a number, as fmaxf)
+__device__ __forceinline__ uint32_t max_bf16x2(uint32_t a, uint32_t b)
+{
+    uint32_t d;
+    asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// (a0 * r, a1 * r), each an IEEE binary32 multiply rounded to nearest even
+__device__ __forceinline__ void mul2_rn(float a0, float a1, float r, float& y0, float& y1)
+{
+    asm("{\n\t.reg .b64 a, b, d;\n\t"
+        "mov.b64 a, {%2, %3};\n\t"
+        "mov.b64 b, {%4, %4};\n\t"
+        "mul.rn.f32x2 d, a, b;\n\t"
+        "mov.b64 {%0, %1}, d;\n\t}"
+        : "=f"(y0), "=f"(y1)
+        : "f"(a0), "f"(a1), "f"(r));
+}
+
 // Encode one block: returns the 8 code bytes (element 2j in the low nibble) and the
-// E4M3 scale byte.
+// E4M3 scale byte.  amax is taken on the bf16 bit patterns (|x| is the pattern with
+// the sign cleared, and the largest |x| is exact in bf16), so it equals the binary32
+// max of |x|; the products x * (1/d) are binary32 multiplies two at a time.
 __device__ __forceinline__ uint2 encode_block(const Block16& b, float g, float t, uint32_t& sb)
 {
-    float f[16];
-    unpack8(b.lo, *reinterpret_cast<float(*)[8]>(&f[0]));
-    unpack8(b.hi, *reinterpret_cast<float(*)[8]>(&f[8]));
-    float amax = 0.0f;
+    const uint32_t v[8] = {b.lo.x, b.lo.y, b.lo.z, b.lo.w, b.hi.x, b.hi.y, b.hi.z, b.hi.w};
+    uint32_t m2 = 0;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[i]));
+    for (int i = 0; i < 8; ++i) m2 = max_bf16x2(m2, v[i] & 0x7FFF7FFFu);
+    m2 = max_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
+    const float amax = __uint_as_float(m2 << 16);
     const float s = (t > 0.0f) ? __fdiv_rn(amax, t) : 0.0f;
     sb = cvt_e4m3x2(s, 0.0f) & 0xFFu;
     const float d = __fmul_rn(e4m3_to_f32(sb), g);
@@ -89,19 +111,45 @@ __device__ __forceinline__ uint2 encode_block(const Block16& b, float g, float t
         const float r = fminf(__frcp_rn(d), FLT_MAX);
         float y[8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[i], r);
+        for (int i = 0; i < 4; ++i)
+            mul2_rn(bf16lo_to_f32(v[i]), bf16hi_to_f32(v[i]), r, y[2 * i], y[2 * i + 1]);
         w.x = cvt_e2m1x8(y);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = __fmul_rn(f[8 + i], r);
+        for (int i = 0; i < 4; ++i)
+            mul2_rn(bf16lo_to_f32(v[4 + i]), bf16hi_to_f32(v[4 + i]), r, y[2 * i], y[2 * i + 1]);
         w.y = cvt_e2m1x8(y);
     }
     return w;
 }
 
+// Division by the blocks per row, n / d for 0 <= n < 2^31, as a multiply-high and a
+// shift (round-up method: with 2^(l-1) < d <= 2^l and m = ceil(2^(31+l) / d), m < 2^32
+// and floor(n*m / 2^(31+l)) = floor(n / d) for every such n).  m == 0 encodes d == 1.
+struct RowDiv {
+    uint32_t m, s;
+};
+
+RowDiv row_div(uint32_t d)
+{
+    RowDiv r{0, 0};
+    if (d <= 1) return r;
+    uint32_t l = 0;
+    while ((uint64_t{1} << l) < d) ++l;
+    const unsigned __int128 num = static_cast<unsigned __int128>(1) << (31 + l);
+    r.m = static_cast<uint32_t>((num + d - 1) / d);
+    r.s = l - 1;
+    return r;
+}
+
+__device__ __forceinline__ uint32_t div_rows(uint32_t n, RowDiv r)
+{
+    return r.m ? (__umulhi(n, r.m) >> r.s) : n;
+}
+
 template <int LAYOUT>
 __device__ __forceinline__ void store_block(uint2* codes, uint8_t* scales, int64_t blk,
                                             int64_t nblk, int64_t nb_row, int64_t kb4, uint2 w,
-                                            uint32_t sb, int lane)
+                                            uint32_t sb, int lane, RowDiv rd, bool idx32)
 {
     // gather 4 consecutive blocks' scale bytes into lane 4j
     const uint32_t s1 = __shfl_down_sync(0xffffffffu, sb, 1);
@@ -115,7 +163,8 @@ __device__ __forceinline__ void store_block(uint2* codes, uint8_t* scales, int64
             if (LAYOUT == BSP_SF_LINEAR) {
                 off = blk;                                   // [rows][K/16] is the block index
             } else {
-                const int64_t row = blk / nb_row;
+                const int64_t row = idx32 ? static_cast<int64_t>(div_rows(static_cast<uint32_t>(blk), rd))
+                                          : blk / nb_row;
                 off = sf_mma_offset(row, blk - row * nb_row, kb4);
             }
             if (blk + 3 < nblk && (off & 3) == 0) {
@@ -128,9 +177,9 @@ __device__ __forceinline__ void store_block(uint2* codes, uint8_t* scales, int64
     }
 }
 
-template <int LAYOUT>
+template <int LAYOUT, bool IDX32>
 __global__ void __launch_bounds__(kQuantThreads)
-    nvfp4_quant_kernel(const uint4* __restrict__ x, int64_t nblk, int64_t nb_row,
+    nvfp4_quant_kernel(const uint4* __restrict__ x, int64_t nblk, int64_t nb_row, RowDiv rd,
                        const float* __restrict__ gptr, uint2* __restrict__ codes,
                        uint8_t* __restrict__ scales)
 {
@@ -155,9 +204,10 @@ __global__ void __launch_bounds__(kQuantThreads)
         Block16 n1 = load_block(x, next + 32 + lane, nblk);
         uint32_t sb0, sb1;
         const uint2 w0 = encode_block(b0, g, t, sb0);
-        store_block<LAYOUT>(codes, scales, base + lane, nblk, nb_row, kb4, w0, sb0, lane);
+        store_block<LAYOUT>(codes, scales, base + lane, nblk, nb_row, kb4, w0, sb0, lane, rd, IDX32);
         const uint2 w1 = encode_block(b1, g, t, sb1);
-        store_block<LAYOUT>(codes, scales, base + 32 + lane, nblk, nb_row, kb4, w1, sb1, lane);
+        store_block<LAYOUT>(codes, scales, base + 32 + lane, nblk, nb_row, kb4, w1, sb1, lane, rd,
+                            IDX32);
         b0 = n0;
         b1 = n1;
         base = next;
@@ -338,14 +388,21 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
     // at most the resident grid (4 CTAs of 256 threads per SM at 64 registers)
     const int grid = grid_for(nblk, (kQuantThreads / 32) * kQBlocksPerWarp, sms, 4);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const auto* xv = static_cast<const uint4*>(x_bf16);
+    auto* cv = reinterpret_cast<uint2*>(codes);
+    // 32-bit block indices (row by multiply-high) whenever a warp span past the end still
+    // fits; the linear layout needs no row at all
+    const bool idx32 = nblk + static_cast<int64_t>(grid) * kQuantThreads * 2 < (int64_t{1} << 31);
+    const RowDiv rd = row_div(static_cast<uint32_t>(K / 16));
     if (layout == BSP_SF_LINEAR)
-        nvfp4_quant_kernel<BSP_SF_LINEAR><<<grid, kQuantThreads, 0, s>>>(
-            static_cast<const uint4*>(x_bf16), nblk, K / 16, global_scale,
-            reinterpret_cast<uint2*>(codes), scales);
+        nvfp4_quant_kernel<BSP_SF_LINEAR, false><<<grid, kQuantThreads, 0, s>>>(
+            xv, nblk, K / 16, rd, global_scale, cv, scales);
+    else if (idx32)
+        nvfp4_quant_kernel<BSP_SF_MMA, true><<<grid, kQuantThreads, 0, s>>>(
+            xv, nblk, K / 16, rd, global_scale, cv, scales);
     else
-        nvfp4_quant_kernel<BSP_SF_MMA><<<grid, kQuantThreads, 0, s>>>(
-            static_cast<const uint4*>(x_bf16), nblk, K / 16, global_scale,
-            reinterpret_cast<uint2*>(codes), scales);
+        nvfp4_quant_kernel<BSP_SF_MMA, false><<<grid, kQuantThreads, 0, s>>>(
+            xv, nblk, K / 16, rd, global_scale, cv, scales);
     return launch_status();
 }
 

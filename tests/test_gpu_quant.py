@@ -85,6 +85,27 @@ def test_nvfp4_quantizer_special_values():
     assert_nvfp4_equal(x, np.float32(0.0), bsp.SF_LINEAR)
 
 
+def test_nvfp4_quantizer_subnormal_and_infinite_inputs():
+    """bf16 subnormal inputs (no flush to zero anywhere) and +-inf (the block scale
+    saturates to 448, the infinite element to +-6)."""
+    sub = np.float32(2.0 ** -130)                       # bf16 subnormal
+    rows = [[sub * (i - 7) for i in range(16)],          # a block of subnormals only
+            [np.inf] + [0.1 * i for i in range(15)],
+            [-np.inf, 1.0, -2.0, 3.0] + [0.0] * 12,
+            [sub, -sub, 1e-3, -1e-3] + [0.25 * i for i in range(12)]]
+    blocks = np.array(rows, dtype=np.float32)
+    x = torch.from_numpy(np.tile(blocks.reshape(1, -1), (64, 1))).to(torch.bfloat16)
+    assert x.shape == (64, 64)
+    for g in (np.float32(2.0 ** -3), np.float32(2.0 ** -140), np.float32(1.0)):
+        for layout in (bsp.SF_LINEAR, bsp.SF_MMA):
+            assert_nvfp4_equal(x, g, layout)
+    # a tensor of subnormals only: its global scale is itself subnormal in binary32
+    xs = torch.from_numpy(np.tile(blocks[:1], (128, 4))).to(torch.bfloat16)
+    gs = oracle.nvfp4_global_scale(xs)
+    assert 0.0 < float(gs) < 1.2e-38
+    assert_nvfp4_equal(xs, gs, bsp.SF_MMA)
+
+
 @pytest.mark.parametrize("M,K,seed", [(256, 3072, 30), (1000, 3072, 31), (4096, 3072, 32),
                                       (7, 24, 33), (64, 12288, 34), (3, 40000, 35)])
 def test_fp8r_quantizer_bit_exact(M, K, seed):
