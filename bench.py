@@ -146,16 +146,22 @@ def cpu_oracle_sample(wl, rows: int, A=None, W=None):
     A = wl.A() if A is None else A
     W = wl.W() if W is None else W
     bias = wl.bias_vec()
-    gw = oracle.nvfp4_global_scale(W)
-    wc, wsf = oracle.nvfp4_quantize(W, gw)          # offline weight prep, untimed
-    ga = oracle.nvfp4_global_scale(A)               # calibrated input scale, untimed
     rows = min(rows, wl.M)
     idx = torch.from_numpy(np.linspace(0, wl.M - 1, rows).astype(np.int64))
     a_rows = A[idx].contiguous()
     b = None if bias is None else bias.float().numpy().astype(np.float64)
-    t0 = time.perf_counter()
-    ac, asf = oracle.nvfp4_quantize(a_rows, ga)
-    oracle.nvfp4_linear(ac, asf, ga, wc, wsf, gw, b)
+    if wl.scheme == "nvfp4":
+        gw = oracle.nvfp4_global_scale(W)
+        wc, wsf = oracle.nvfp4_quantize(W, gw)          # offline weight prep, untimed
+        ga = oracle.nvfp4_global_scale(A)               # calibrated input scale, untimed
+        t0 = time.perf_counter()
+        ac, asf = oracle.nvfp4_quantize(a_rows, ga)
+        oracle.nvfp4_linear(ac, asf, ga, wc, wsf, gw, b)
+    else:
+        wq, ws = oracle.fp8r_quantize(W)                # offline weight prep, untimed
+        t0 = time.perf_counter()
+        aq, as_ = oracle.fp8r_quantize(a_rows)
+        oracle.fp8r_linear(aq, as_, wq, ws, b)
     dt = time.perf_counter() - t0
     return dt, 2.0 * rows * wl.N * wl.K, oracle.default_threads()
 
@@ -215,8 +221,7 @@ def run_bsp(args):
                                 device_id=dev)
 
     wl = synth.WORKLOADS[args.workload]
-    if wl.scheme != "nvfp4":
-        raise SystemExit(f"workload {wl.name} is not an NVFP4 linear")
+    nvf4 = wl.scheme == "nvfp4"
     M, N, K = wl.M, wl.N, wl.K
     A_cpu = wl.A()
     A_host = A_cpu.pin_memory()
@@ -225,28 +230,45 @@ def run_bsp(args):
     bias = wl.bias_vec()
     bias = None if bias is None else bias.to(dev)
 
-    # untimed preparation: pre-quantized weights and a calibrated activation scale
-    gw = bsp.nvfp4_global_scale(W)
-    wc, wsf = bsp.nvfp4_quantize_act(W, gw, layout=bsp.SF_MMA)
-    ga = bsp.nvfp4_global_scale(A)
-    ac = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
-    asf = torch.empty((bsp.nvfp4_sf_bytes(M, K, bsp.SF_MMA),), dtype=torch.uint8, device=dev)
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
     y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    if nvf4:
+        # untimed preparation: pre-quantized weights and a calibrated activation scale
+        gw = bsp.nvfp4_global_scale(W)
+        wc, wsf = bsp.nvfp4_quantize_act(W, gw, layout=bsp.SF_MMA)
+        ga = bsp.nvfp4_global_scale(A)
+        ac = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        asf = torch.empty((bsp.nvfp4_sf_bytes(M, K, bsp.SF_MMA),), dtype=torch.uint8, device=dev)
+        ws = torch.empty((bsp.nvfp4_linear_workspace_bytes(M, K),), dtype=torch.uint8,
+                         device=dev)
 
-    ws = torch.empty((bsp.nvfp4_linear_workspace_bytes(M, K),), dtype=torch.uint8, device=dev)
+        def quant():
+            bsp.nvfp4_quantize_act(A, ga, codes=ac, scales=asf, layout=bsp.SF_MMA)
 
-    def quant():
-        bsp.nvfp4_quantize_act(A, ga, codes=ac, scales=asf, layout=bsp.SF_MMA)
+        def gemm():
+            bsp.nvfp4_gemm(ac, asf, ga, wc, wsf, gw, bias=bias, out=y)
 
-    def gemm():
-        bsp.nvfp4_gemm(ac, asf, ga, wc, wsf, gw, bias=bias, out=y)
+        def step():
+            # the whole path in one call: quantizer, then the GEMM as its programmatic
+            # dependent
+            bsp.nvfp4_linear(A, ga, wc, wsf, gw, bias=bias, out=y, workspace=ws)
+    else:
+        # untimed preparation: the weight quantized once per row
+        wq, wsc = bsp.fp8r_quantize_rows(W)
+        aq = torch.empty((M, K), dtype=torch.uint8, device=dev)
+        asc = torch.empty((M,), dtype=torch.float32, device=dev)
 
-    def step():
-        # the whole path in one call: quantizer, then the GEMM as its programmatic dependent
-        bsp.nvfp4_linear(A, ga, wc, wsf, gw, bias=bias, out=y, workspace=ws)
+        def quant():
+            bsp.fp8r_quantize_rows(A, q=aq, row_scale=asc)
+
+        def gemm():
+            bsp.fp8r_gemm(aq, asc, wq, wsc, bias=bias, out=y)
+
+        def step():
+            quant()
+            gemm()
 
     quant()
     gemm()
@@ -334,8 +356,14 @@ def run_bsp(args):
     g_mean = statistics.mean(g_ms)
     pk, pk_src = peaks()
     hbm = pk["hbm_gbs"]
-    fp4_peak = 4.0 * pk["bf16_tflops"]          # nominal fp4 : bf16 dense ratio = 9 : 2.25
-    q_bytes = M * K * 2.5625                    # 2 B read + 0.5 B codes + 1/16 B scales per element
+    if nvf4:
+        q_bytes = M * K * 2.5625                # 2 B read + 0.5 B codes + 1/16 B scales per element
+        mm_peak = 4.0 * pk["bf16_tflops"]       # nominal dense fp4 : bf16 = 9 : 2.25
+    else:
+        q_bytes = M * K * 3.0 + 4.0 * M         # 2 B read + 1 B code per element + a row scale
+        mm_peak = 2.0 * pk["bf16_tflops"]       # nominal dense fp8 : bf16 = 4.5 : 2.25
+    qname = "nvfp4_quantize_act" if nvf4 else "fp8r_quantize_rows"
+    gname = "nvfp4_gemm" if nvf4 else "fp8r_gemm"
     gemm_tflops = flops / (g_mean * 1e-3) / 1e12
     q_gbs = q_bytes / (q_mean * 1e-3) / 1e9
     traffic = ncu_traffic(wl.name)
@@ -345,23 +373,25 @@ def run_bsp(args):
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "vs_baseline": None, "dtype": "nvfp4" if nvf4 else "fp8_e4m3", "data": "synthetic",
         "config": {"workload": wl.name, "M": M, "N": N, "K": K, "bias": wl.bias,
-                   "step": "nvfp4_linear = nvfp4_quantize_act + nvfp4_gemm (fused alpha, "
-                           "bias, bf16; GEMM as programmatic dependent), one CUDA graph",
+                   "step": ("nvfp4_linear = nvfp4_quantize_act + nvfp4_gemm (fused alpha, "
+                            "bias, bf16; GEMM as programmatic dependent), one CUDA graph")
+                   if nvf4 else ("fp8r_quantize_rows + fp8r_gemm (fused row scales, bias, "
+                                 "bf16), one CUDA graph"),
                    "l2": "flushed before every step (256 MiB write, outside the events)",
                    "parallelism": "replicas" if world > 1 else "single"},
-        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": fp4_peak,
-                     "unit": "TFLOP/s", "frac": gemm_tflops / fp4_peak, "traffic": traffic,
-                     "kernel": "nvfp4_gemm",
-                     "peak_source": f"{pk_src}: 4 x bf16 burst {pk['bf16_tflops']} TFLOP/s "
-                                    "(nominal dense fp4:bf16 = 4)"},
+        "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": mm_peak,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / mm_peak, "traffic": traffic,
+                     "kernel": gname,
+                     "peak_source": f"{pk_src}: {4 if nvf4 else 2} x bf16 burst "
+                                    f"{pk['bf16_tflops']} TFLOP/s (nominal dense "
+                                    f"{'fp4' if nvf4 else 'fp8'}:bf16 = {4 if nvf4 else 2})"},
         "kernels": {
-            "nvfp4_quantize_act": {"us": 1e3 * q_mean, "GB/s": q_gbs, "frac_hbm": q_gbs / hbm,
-                                   "bytes": q_bytes, "hbm_peak": hbm},
-            "nvfp4_gemm": {"us": 1e3 * g_mean, "TFLOP/s": gemm_tflops,
-                           "frac_fp4": gemm_tflops / fp4_peak,
-                           "frac_fp4_datasheet": gemm_tflops / 9000.0},
+            qname: {"us": 1e3 * q_mean, "GB/s": q_gbs, "frac_hbm": q_gbs / hbm,
+                    "bytes": q_bytes, "hbm_peak": hbm},
+            gname: {"us": 1e3 * g_mean, "TFLOP/s": gemm_tflops, "frac_peak": gemm_tflops / mm_peak,
+                    "frac_datasheet": gemm_tflops / (9000.0 if nvf4 else 4500.0)},
         },
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
