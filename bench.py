@@ -51,6 +51,15 @@ def parse():
     p.add_argument("--impl", choices=["bsp", "reference"], default="bsp")
     p.add_argument("--workload", default="nvfp4_attn_1mp")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--m", type=int, default=0,
+                   help="token count (rows of A) instead of the workload's own, e.g. the fp8r "
+                        "sweep 256 / 1024 / 16384")
+    p.add_argument("--chain", nargs="?", const="fused", default=None,
+                   choices=["fused", "unfused"],
+                   help="MLP workloads: time the up projection, the re-quantization of its output "
+                        "and the down projection as one step; 'fused' (default) re-quantizes in "
+                        "the up projection's epilogue (nvfp4_gemm_quant), 'unfused' writes bf16 "
+                        "and runs the quantizer on it")
     p.add_argument("--cpu-rows", type=int, default=2048,
                    help="rows of A in the CPU-oracle baseline sample")
     return p.parse_args()
@@ -146,8 +155,9 @@ def cpu_oracle_sample(wl, rows: int, A=None, W=None):
     A = wl.A() if A is None else A
     W = wl.W() if W is None else W
     bias = wl.bias_vec()
-    rows = min(rows, wl.M)
-    idx = torch.from_numpy(np.linspace(0, wl.M - 1, rows).astype(np.int64))
+    m_total = A.shape[0]
+    rows = min(rows, m_total)
+    idx = torch.from_numpy(np.linspace(0, m_total - 1, rows).astype(np.int64))
     a_rows = A[idx].contiguous()
     b = None if bias is None else bias.float().numpy().astype(np.float64)
     if wl.scheme == "nvfp4":
@@ -172,7 +182,8 @@ def run_reference(args):
         return 0
     import synth
     wl = synth.WORKLOADS[args.workload]
-    A, W = wl.A(), wl.W()
+    M = args.m if args.m else wl.M
+    A, W = (wl.A() if M == wl.M else wl.A_rows(M)), wl.W()
     # size each step's sample so the whole run stays within a few minutes
     dt, _, _ = cpu_oracle_sample(wl, 16, A, W)
     budget_s = 150.0 / max(1, args.steps + args.warmup)
@@ -185,14 +196,14 @@ def run_reference(args):
         tot += dt
         flops += fl
     value = flops / tot / 1e12
-    sample = (f"{rows} of {wl.M} rows of A per step (quantize + fp64 GEMM against the "
+    sample = (f"{rows} of {M} rows of A per step (quantize + fp64 GEMM against the "
               f"full {wl.N}x{wl.K} weight); weight quantization untimed")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * tot / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.M, "N": wl.N, "K": wl.K, "bias": wl.bias,
+        "config": {"workload": wl.name, "M": M, "N": wl.N, "K": wl.K, "bias": wl.bias,
                    "sample_rows": rows},
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
                          "sample": sample},
@@ -222,18 +233,26 @@ def run_bsp(args):
 
     wl = synth.WORKLOADS[args.workload]
     nvf4 = wl.scheme == "nvfp4"
-    M, N, K = wl.M, wl.N, wl.K
-    A_cpu = wl.A()
+    if args.chain and not wl.name.startswith("nvfp4_mlp"):
+        raise SystemExit("--chain applies to the NVFP4 MLP workloads")
+    M = args.m if args.m else wl.M
+    N, K = wl.N, wl.K
+    A_cpu = wl.A() if M == wl.M else wl.A_rows(M)
     A_host = A_cpu.pin_memory()
     A = A_cpu.to(dev)
     W = wl.W().to(dev)
     bias = wl.bias_vec()
     bias = None if bias is None else bias.to(dev)
+    pk, pk_src = peaks()
+    hbm = pk["hbm_gbs"]
+    mm_peak = (4.0 if nvf4 else 2.0) * pk["bf16_tflops"]   # nominal dense fp4 / fp8 : bf16
 
     y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
-    y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
     flush = torch.empty((L2_FLUSH_BYTES,), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
+    # per-kernel parts in step order: (name, fn, unit, algorithmic work per launch, peak)
+    parts = []
+    flops = 2.0 * M * N * K
     if nvf4:
         # untimed preparation: pre-quantized weights and a calibrated activation scale
         gw = bsp.nvfp4_global_scale(W)
@@ -241,49 +260,76 @@ def run_bsp(args):
         ga = bsp.nvfp4_global_scale(A)
         ac = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
         asf = torch.empty((bsp.nvfp4_sf_bytes(M, K, bsp.SF_MMA),), dtype=torch.uint8, device=dev)
-        ws = torch.empty((bsp.nvfp4_linear_workspace_bytes(M, K),), dtype=torch.uint8,
+        ws = torch.empty((bsp.nvfp4_linear_workspace_bytes(M, max(K, N)),), dtype=torch.uint8,
                          device=dev)
-
-        def quant():
-            bsp.nvfp4_quantize_act(A, ga, codes=ac, scales=asf, layout=bsp.SF_MMA)
-
-        def gemm():
-            bsp.nvfp4_gemm(ac, asf, ga, wc, wsf, gw, bias=bias, out=y)
-
-        def step():
-            # the whole path in one call: quantizer, then the GEMM as its programmatic
-            # dependent
-            bsp.nvfp4_linear(A, ga, wc, wsf, gw, bias=bias, out=y, workspace=ws)
+        parts.append(("nvfp4_quantize_act", lambda: bsp.nvfp4_quantize_act(
+            A, ga, codes=ac, scales=asf, layout=bsp.SF_MMA), "GB/s", M * K * 2.5625, hbm))
+        parts.append(("nvfp4_gemm", lambda: bsp.nvfp4_gemm(
+            ac, asf, ga, wc, wsf, gw, bias=bias, out=y), "TFLOP/s", flops, mm_peak))
+        # the whole path in one call: quantizer, then the GEMM as its programmatic dependent
+        step_fns = [lambda: bsp.nvfp4_linear(A, ga, wc, wsf, gw, bias=bias, out=y, workspace=ws)]
+        y_out = y
+        if args.chain:
+            # MLP down projection on GEMM1's output: a6 re-quantizes it with a scale
+            # calibrated (once, untimed) on that output, then GEMM2 [M, K] = Y1 . W2^T
+            W2 = wl.W2().to(dev)
+            g2w = bsp.nvfp4_global_scale(W2)
+            w2c, w2sf = bsp.nvfp4_quantize_act(W2, g2w, layout=bsp.SF_MMA)
+            step_fns[0]()
+            g2 = bsp.nvfp4_global_scale(y)
+            y1c = torch.empty((M, N // 2), dtype=torch.uint8, device=dev)
+            y1sf = torch.empty((bsp.nvfp4_sf_bytes(M, N, bsp.SF_MMA),), dtype=torch.uint8,
+                               device=dev)
+            y2 = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+            gemm2 = ("nvfp4_gemm (down)", lambda: bsp.nvfp4_gemm(
+                y1c, y1sf, g2, w2c, w2sf, g2w, out=y2), "TFLOP/s", 2.0 * M * K * N, mm_peak)
+            if args.chain == "fused":
+                # up projection with the re-quantization in its epilogue: no bf16 Y1
+                up_q = ("nvfp4_gemm_quant (up + a6 in the epilogue)", lambda: bsp.nvfp4_gemm_quant(
+                    ac, asf, ga, wc, wsf, gw, g2, bias=bias, out_codes=y1c, out_sf=y1sf),
+                    "TFLOP/s", flops, mm_peak)
+                parts[1] = up_q
+                parts.append(gemm2)
+                step_fns = [parts[0][1], up_q[1], gemm2[1]]
+            else:
+                parts.append(("nvfp4_quantize_act (a6, on GEMM1's output)", lambda: bsp.nvfp4_quantize_act(
+                    y, g2, codes=y1c, scales=y1sf, layout=bsp.SF_MMA), "GB/s", M * N * 2.5625, hbm))
+                parts.append(gemm2)
+                step_fns.append(lambda: bsp.nvfp4_linear(y, g2, w2c, w2sf, g2w, out=y2,
+                                                         workspace=ws))
+            flops += 2.0 * M * K * N
+            y_out = y2
     else:
         # untimed preparation: the weight quantized once per row
         wq, wsc = bsp.fp8r_quantize_rows(W)
         aq = torch.empty((M, K), dtype=torch.uint8, device=dev)
         asc = torch.empty((M,), dtype=torch.float32, device=dev)
+        parts.append(("fp8r_quantize_rows", lambda: bsp.fp8r_quantize_rows(
+            A, q=aq, row_scale=asc), "GB/s", M * K * 3.0 + 4.0 * M, hbm))
+        parts.append(("fp8r_gemm", lambda: bsp.fp8r_gemm(
+            aq, asc, wq, wsc, bias=bias, out=y), "TFLOP/s", flops, mm_peak))
+        step_fns = [parts[0][1], parts[1][1]]
+        y_out = y
+    y_host = torch.empty(tuple(y_out.shape), dtype=torch.bfloat16).pin_memory()
 
-        def quant():
-            bsp.fp8r_quantize_rows(A, q=aq, row_scale=asc)
+    def step():
+        for f in step_fns:
+            f()
 
-        def gemm():
-            bsp.fp8r_gemm(aq, asc, wq, wsc, bias=bias, out=y)
-
-        def step():
-            quant()
-            gemm()
-
-    quant()
-    gemm()
+    for p in parts:
+        p[1]()
     step()
     torch.cuda.synchronize(dev)
     if bsp.bsp_last_device_status() != 0:
         raise SystemExit("device status not OK after the first step")
-    gq, gg, gs = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+    graphs = [torch.cuda.CUDAGraph() for _ in parts]
+    gs = torch.cuda.CUDAGraph()
     side = torch.cuda.Stream(dev)
     side.wait_stream(stream)
     with torch.cuda.stream(side):
-        with torch.cuda.graph(gq, stream=side):
-            quant()
-        with torch.cuda.graph(gg, stream=side):
-            gemm()
+        for g, p in zip(graphs, parts):
+            with torch.cuda.graph(g, stream=side):
+                p[1]()
         with torch.cuda.graph(gs, stream=side):
             step()
     stream.wait_stream(side)
@@ -306,30 +352,31 @@ def run_bsp(args):
             gs.replay()
             ev[i][1].record(stream)
         torch.cuda.synchronize(dev)
+        # per-kernel split (roofline of each kernel): the same kernels in step order,
+        # each replayed from its own graph, the L2 flushed before each sequence
+        kev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(parts) + 1)]
+               for _ in range(n_ev)]
+        for i in range(args.steps):
+            flush.fill_(1)
+            kev[i][0].record(stream)
+            for j, g in enumerate(graphs):
+                g.replay()
+                kev[i][j + 1].record(stream)
+        torch.cuda.synchronize(dev)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize(dev)
     s_ms = [e[0].elapsed_time(e[1]) for e in ev]
     total_ms = sum(s_ms)
-    # per-kernel split (roofline of each kernel): the same kernels, each its own graph
-    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_ev)]
-    for i in range(args.steps):
-        flush.fill_(1)
-        kev[i][0].record(stream)
-        gq.replay()
-        kev[i][1].record(stream)
-        gg.replay()
-        kev[i][2].record(stream)
-    torch.cuda.synchronize(dev)
-    q_ms = [e[0].elapsed_time(e[1]) for e in kev]
-    g_ms = [e[1].elapsed_time(e[2]) for e in kev]
+    part_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in kev)
+               for j in range(len(parts))]
     if world > 1:
         t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         total_ms = float(t.item())
     if bsp.bsp_last_device_status() != 0:
         raise SystemExit("device status not OK after the timed steps")
-    if not torch.isfinite(y.float()).all():
+    if not torch.isfinite(y_out.float()).all():
         raise SystemExit("non-finite output")
 
     # end to end through the public API: pinned host A in, host Y out, every step
@@ -341,7 +388,7 @@ def run_bsp(args):
             e0.record(stream)
         A.copy_(A_host, non_blocking=True)
         step()
-        y_host.copy_(y, non_blocking=True)
+        y_host.copy_(y_out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
@@ -350,23 +397,25 @@ def run_bsp(args):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         e2e_ms = float(t.item())
 
-    flops = 2.0 * M * N * K
     ms_per_step = total_ms / args.steps
-    q_mean = statistics.mean(q_ms)
-    g_mean = statistics.mean(g_ms)
-    pk, pk_src = peaks()
-    hbm = pk["hbm_gbs"]
+    kernels = {}
+    for (name, _, unit, work, peak), ms in zip(parts, part_ms):
+        rate = work / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
+        kernels[name] = {"us": 1e3 * ms, unit: rate, "frac_peak": rate / peak, "peak": peak,
+                         "work_per_launch": work}
+    gname, _, _, _, _ = parts[1]
+    gemm_tflops = kernels[gname]["TFLOP/s"]
     if nvf4:
-        q_bytes = M * K * 2.5625                # 2 B read + 0.5 B codes + 1/16 B scales per element
-        mm_peak = 4.0 * pk["bf16_tflops"]       # nominal dense fp4 : bf16 = 9 : 2.25
+        step_desc = ("nvfp4_linear = nvfp4_quantize_act + nvfp4_gemm (fused alpha, bias, bf16; "
+                     "GEMM as programmatic dependent)")
+        if args.chain == "fused":
+            step_desc = ("nvfp4_quantize_act + nvfp4_gemm_quant (up projection, its output "
+                         "re-quantized in the epilogue) + nvfp4_gemm (down projection), each "
+                         "GEMM a programmatic dependent of the kernel before it")
+        elif args.chain == "unfused":
+            step_desc += "; then nvfp4_linear of GEMM1's bf16 output through the down projection"
     else:
-        q_bytes = M * K * 3.0 + 4.0 * M         # 2 B read + 1 B code per element + a row scale
-        mm_peak = 2.0 * pk["bf16_tflops"]       # nominal dense fp8 : bf16 = 4.5 : 2.25
-    qname = "nvfp4_quantize_act" if nvf4 else "fp8r_quantize_rows"
-    gname = "nvfp4_gemm" if nvf4 else "fp8r_gemm"
-    gemm_tflops = flops / (g_mean * 1e-3) / 1e12
-    q_gbs = q_bytes / (q_mean * 1e-3) / 1e9
-    traffic = ncu_traffic(wl.name)
+        step_desc = "fp8r_quantize_rows + fp8r_gemm (fused row scales, bias, bf16)"
     line = {
         "metric": METRIC,
         "value": world * flops / (ms_per_step * 1e-3) / 1e12,
@@ -375,38 +424,32 @@ def run_bsp(args):
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "nvfp4" if nvf4 else "fp8_e4m3", "data": "synthetic",
         "config": {"workload": wl.name, "M": M, "N": N, "K": K, "bias": wl.bias,
-                   "step": ("nvfp4_linear = nvfp4_quantize_act + nvfp4_gemm (fused alpha, "
-                            "bias, bf16; GEMM as programmatic dependent), one CUDA graph")
-                   if nvf4 else ("fp8r_quantize_rows + fp8r_gemm (fused row scales, bias, "
-                                 "bf16), one CUDA graph"),
+                   "chain": args.chain, "step": step_desc + ", one CUDA graph",
                    "l2": "flushed before every step (256 MiB write, outside the events)",
                    "parallelism": "replicas" if world > 1 else "single"},
         "roofline": {"bound": "tensor", "achieved": gemm_tflops, "peak": mm_peak,
-                     "unit": "TFLOP/s", "frac": gemm_tflops / mm_peak, "traffic": traffic,
+                     "unit": "TFLOP/s", "frac": gemm_tflops / mm_peak,
+                     "traffic": ncu_traffic(wl.name) if M == wl.M else None,
                      "kernel": gname,
                      "peak_source": f"{pk_src}: {4 if nvf4 else 2} x bf16 burst "
                                     f"{pk['bf16_tflops']} TFLOP/s (nominal dense "
                                     f"{'fp4' if nvf4 else 'fp8'}:bf16 = {4 if nvf4 else 2})"},
-        "kernels": {
-            qname: {"us": 1e3 * q_mean, "GB/s": q_gbs, "frac_hbm": q_gbs / hbm,
-                    "bytes": q_bytes, "hbm_peak": hbm},
-            gname: {"us": 1e3 * g_mean, "TFLOP/s": gemm_tflops, "frac_peak": gemm_tflops / mm_peak,
-                    "frac_datasheet": gemm_tflops / (9000.0 if nvf4 else 4500.0)},
-        },
+        "kernels": kernels,
         "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": M * N * 2},
-        "gpu_launches": 2 * args.steps,
+                "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": y_out.numel() * 2},
+        "gpu_launches": len(parts) * args.steps,
         "clocks": sampler.summary(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         dt, fl, cores = cpu_oracle_sample(wl, args.cpu_rows, A_cpu)
         line["cpu_baseline"] = {
             "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-            "sample": f"{args.cpu_rows} of {M} rows of A: quantize + fp64 GEMM against the "
-                      f"full weight ({dt:.1f} s)"}
+            "sample": f"{min(args.cpu_rows, M)} of {M} rows of A: quantize + fp64 GEMM "
+                      f"against the full weight ({dt:.1f} s)"
+                      + ("; first linear of the chain only" if args.chain else "")}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del gq, gg, gs
+    del graphs, gs
     if world > 1:
         dist.destroy_process_group()
     return 0

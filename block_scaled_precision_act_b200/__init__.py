@@ -20,7 +20,7 @@ import torch
 
 __all__ = [
     "BSPError", "SF_LINEAR", "SF_MMA", "lib", "library_path",
-    "nvfp4_quantize_act", "nvfp4_gemm", "fp8r_quantize_rows", "fp8r_gemm",
+    "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_quant", "fp8r_quantize_rows", "fp8r_gemm",
     "nvfp4_linear", "nvfp4_linear_workspace_bytes", "nvfp4_linear_noalloc",
     "nvfp4_linear_noalloc_max_bytes",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
@@ -42,6 +42,8 @@ _SIGS = {
     "nvfp4_quantize_act": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp, _c_int, _c_vp], _c_int),
     "nvfp4_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                     _c_i64, _c_vp], _c_int),
+    "nvfp4_gemm_quant": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp,
+                          _c_i64, _c_i64, _c_i64, _c_vp], _c_int),
     "nvfp4_linear": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64,
                       _c_vp, _c_i64, _c_vp], _c_int),
     "nvfp4_linear_workspace_bytes": ([_c_i64, _c_i64], _c_i64),
@@ -167,6 +169,26 @@ def nvfp4_gemm(a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias=None, out=
                             _ptr(w_sf), _ptr(w_global), _ptr(bias), _ptr(out), M, N, 2 * K2,
                             _stream(stream)))
     return out
+
+
+def nvfp4_gemm_quant(a_codes, a_sf, a_global, w_codes, w_sf, w_global, out_global, bias=None,
+                     out_codes=None, out_sf=None, stream=None):
+    """nvfp4_gemm whose bf16 output is re-quantized in the epilogue for the next nvfp4
+    linear: returns (codes uint8 [M, N/2], MMA-layout scales) under `out_global`."""
+    M, K2 = a_codes.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] != K2:
+        raise BSPError("nvfp4_gemm_quant (K mismatch)", -1)
+    if out_codes is None:
+        out_codes = torch.empty((M, N // 2), dtype=torch.uint8, device=a_codes.device)
+    if out_sf is None:
+        out_sf = torch.empty((max(nvfp4_sf_bytes(M, N, SF_MMA), 0),), dtype=torch.uint8,
+                             device=a_codes.device)
+    _check("nvfp4_gemm_quant",
+           lib().nvfp4_gemm_quant(_ptr(a_codes), _ptr(a_sf), _ptr(a_global), _ptr(w_codes),
+                                  _ptr(w_sf), _ptr(w_global), _ptr(bias), _ptr(out_global),
+                                  _ptr(out_codes), _ptr(out_sf), M, N, 2 * K2, _stream(stream)))
+    return out_codes, out_sf
 
 
 def nvfp4_linear_workspace_bytes(M: int, K: int) -> int:

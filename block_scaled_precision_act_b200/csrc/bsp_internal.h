@@ -17,14 +17,6 @@ int* device_status_ptr(int device);
 // Bounded-wait limit for kernels, in nanoseconds.
 uint64_t wait_limit_ns();
 
-// nvfp4_gemm launched with programmatic stream serialisation: for a GEMM whose A codes
-// and scales are written by the kernel launched just before it on the same stream (the
-// activation quantizer).  Same arguments, checks and results as nvfp4_gemm.
-int nvfp4_gemm_dependent(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
-                         const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
-                         const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
-                         bsp_stream_t stream);
-
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int launch_status()

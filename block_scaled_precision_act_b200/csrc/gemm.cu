@@ -36,6 +36,7 @@
 #include "bsp_internal.h"
 #include "bsp_ptx.cuh"
 #include "bsp_testing.h"
+#include "nvfp4_block.cuh"
 
 namespace bsp {
 namespace {
@@ -56,6 +57,10 @@ struct GemmArgs {
     int* status;                     // device status word
     uint64_t wait_ns;                // bounded-wait limit
     int64_t debug_stop_iter;         // < 0 in normal use; test hook, see bsp_testing.h
+    // output re-quantized to NVFP4 instead of written as bf16 (pair kernel, QOUT):
+    const float* q_global;           // device fp32 global scale g of the next layer
+    uint8_t* q_codes;                // [M][N/2] E2M1 codes of bf16(Y)
+    uint8_t* q_sf;                   // E4M3 block scales of bf16(Y), MMA layout, K = N
 };
 
 template <bool NVF4, int BN, int STAGES, int NACC>
@@ -100,6 +105,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs args)
 {
+    griddep_launch_dependents();   // a dependent grid may start its prologue meanwhile
     using C = Cfg<NVF4, BN, STAGES, NACC>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -264,7 +270,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int q = warp & 3;                 // TMEM lane quadrant of this warp
         const int row_in_tile = q * 32 + lane;
         float alpha = 0.0f;
-        if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
         int acc_it = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
             const int mt = tile % num_m, nt = tile / num_m;
@@ -273,6 +278,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool ok = mbar_wait(tfull + a, aph, abort_flag, args.wait_ns, args.status, 4);
             if (!__all_sync(0xffffffffu, ok)) break;   // also reconverges the warp
             tc_fence_after();
+            // read here, after the producer's griddep_wait (through the accumulator
+            // barrier), so a preceding grid may still be writing the scales at launch
+            if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
             const int m = mt * kBM + row_in_tile;
             float sa = 0.0f;
             if constexpr (!NVF4) sa = (m < M) ? __ldg(args.a_scale + m) : 0.0f;
@@ -406,7 +414,7 @@ struct PairCfg {
     static_assert(!NVF4 || ATOMS == 1, "scale copies are staged per atom");
 };
 
-template <bool NVF4>
+template <bool NVF4, bool QOUT>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREADS, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                      const __grid_constant__ CUtensorMap tmB,
@@ -414,6 +422,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                      const __grid_constant__ CUtensorMap tmSFB,
                      const __grid_constant__ CUtensorMap tmY, const GemmArgs args)
 {
+    static_assert(NVF4 || !QOUT, "the re-quantized output is NVFP4 only");
+    griddep_launch_dependents();   // a dependent grid may start its prologue meanwhile
     using C = PairCfg<NVF4>;
     constexpr int STAGES = C::STAGES;
     extern __shared__ uint8_t smem_raw[];
@@ -635,7 +645,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
         uint8_t* slab0 = sEpi + ew * 2 * C::EPI_SLAB;
         float alpha = 0.0f;
-        if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
+        float qg = 0.0f, qt = 0.0f;      // re-quantization: g of the next layer and 6g
+        const int64_t q_kb4 = N / 64;
         int acc_it = 0;
         int buf = 0;
         int committed = 0;               // bulk-store groups this warp committed
@@ -647,6 +658,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                                       args.wait_ns, args.status, 14);
             if (!__all_sync(0xffffffffu, ok)) break;   // also reconverges the warp
             tc_fence_after();
+            // read here, after the producer's griddep_wait (through the accumulator
+            // barrier), so a preceding grid may still be writing the scales at launch
+            if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
+            if constexpr (QOUT) {
+                qg = __ldg(args.q_global);
+                qt = __fmul_rn(6.0f, qg);
+            }
             const int sacc = acc_it & 1;
             const int wrow = mt * 256 + static_cast<int>(rank) * 128 + q * 32;   // warp's first row
             const int m = wrow + lane;
@@ -716,6 +734,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     }
 #pragma unroll
                     for (int i = 0; i < 4; ++i) packed[g * 4 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                }
+                if constexpr (QOUT) {
+                    // bf16(Y) re-quantized in registers: this lane's 32 columns are two
+                    // whole 16-element blocks of row m (N % 64 == 0)
+                    if (m < M && n0 < N) {
+                        const uint32_t b0[8] = {packed[0], packed[1], packed[2], packed[3],
+                                                packed[4], packed[5], packed[6], packed[7]};
+                        const uint32_t b1[8] = {packed[8], packed[9], packed[10], packed[11],
+                                                packed[12], packed[13], packed[14], packed[15]};
+                        uint32_t sb0, sb1;
+                        const uint2 c0 = nvfp4_encode_block16(b0, qg, qt, sb0);
+                        const uint2 c1 = nvfp4_encode_block16(b1, qg, qt, sb1);
+                        *reinterpret_cast<uint4*>(args.q_codes + static_cast<int64_t>(m) * (N / 2) +
+                                                  n0 / 2) = make_uint4(c0.x, c0.y, c1.x, c1.y);
+                        *reinterpret_cast<uint16_t*>(args.q_sf +
+                                                     sf_mma_offset(m, n0 / 16, q_kb4)) =
+                            static_cast<uint16_t>(sb0 | (sb1 << 8));
+                    }
+                    continue;
                 }
                 // the TMA store that last read this slab must be done reading it
                 if (lane == 0 && last_group[buf] >= 0) {
@@ -868,7 +905,7 @@ cudaError_t launch_kernel(void (*kernel)(Params...), unsigned grid, unsigned blo
     return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <bool NVF4>
+template <bool NVF4, bool QOUT = false>
 int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, int sms,
                 cudaStream_t s, bool pdl)
 {
@@ -877,7 +914,7 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
     static cudaError_t err[64];
     static int max_pairs[64];
     std::call_once(once[dev], [&] {
-        err[dev] = cudaFuncSetAttribute(gemm_pair_kernel<NVF4>,
+        err[dev] = cudaFuncSetAttribute(gemm_pair_kernel<NVF4, QOUT>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
         max_pairs[dev] = sms / 2;
         if (err[dev] == cudaSuccess) {
@@ -893,7 +930,7 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
             cfg.attrs = attr;
             cfg.numAttrs = 1;
             int clusters = 0;
-            if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<NVF4>, &cfg) ==
+            if (cudaOccupancyMaxActiveClusters(&clusters, gemm_pair_kernel<NVF4, QOUT>, &cfg) ==
                     cudaSuccess &&
                 clusters > 0)
                 max_pairs[dev] = clusters < sms / 2 ? clusters : sms / 2;
@@ -914,7 +951,9 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
         if (st == BSP_OK)
             st = make_map_atoms(&tmB, w, row_bytes, static_cast<uint64_t>(args.N), C::ATOMS);
     }
-    if (st == BSP_OK)
+    if (QOUT)
+        std::memset(&tmY, 0, sizeof(tmY));      // no bf16 output: the map is never used
+    else if (st == BSP_OK)
         st = make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, args.out,
                          static_cast<uint64_t>(args.N), static_cast<uint64_t>(args.M), 32, 32,
                          CU_TENSOR_MAP_SWIZZLE_64B);
@@ -933,8 +972,8 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
     const int64_t tiles =
         static_cast<int64_t>((args.M + 255) / 256) * ((args.N + 255) / 256);
     const int pairs = static_cast<int>(tiles < max_pairs[dev] ? tiles : max_pairs[dev]);
-    if (launch_kernel(gemm_pair_kernel<NVF4>, 2 * pairs, C::THREADS, C::SMEM_BYTES, s, pdl, tmA,
-                      tmB, tmSFA, tmSFB, tmY, args) != cudaSuccess) {
+    if (launch_kernel(gemm_pair_kernel<NVF4, QOUT>, 2 * pairs, C::THREADS, C::SMEM_BYTES, s, pdl,
+                      tmA, tmB, tmSFA, tmSFB, tmY, args) != cudaSuccess) {
         cudaGetLastError();
         return BSP_ERR_CUDA;
     }
@@ -1003,14 +1042,33 @@ int check_gemm_common(const void* a, const void* w, const void* bias, const void
     return BSP_OK;
 }
 
+// NVFP4 re-quantization of the output (nvfp4_gemm_quant) instead of a bf16 Y
+struct QOut {
+    const float* global;
+    uint8_t* codes;
+    uint8_t* sf;
+};
+
+// Every launch allows programmatic stream serialisation: the kernels read no input and
+// write no output before their producer's griddep_wait() (the epilogue's reads and
+// writes follow it through the pipeline barriers), so a preceding grid that triggers
+// early only lets the prologue overlap its tail, and one that does not (any other
+// library's kernel) completes first as usual.
 int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_scale,
                const uint8_t* w, const uint8_t* sfb, const float* w_scale, const void* bias,
                void* out, int64_t M, int64_t N, int64_t K, bsp_stream_t stream,
-               int64_t debug_stop_iter, uint64_t wait_ns_override, bool pdl)
+               int64_t debug_stop_iter, uint64_t wait_ns_override, const QOut* q = nullptr)
 {
-    int st = check_gemm_common(a, w, bias, out, M, N, K);
+    const bool pdl = true;
+    int st = check_gemm_common(a, w, bias, q ? static_cast<void*>(q->codes) : out, M, N, K);
     if (st != BSP_OK || M == 0 || N == 0) return st;
     if (!a_scale || !w_scale) return BSP_ERR_INVALID_ARG;
+    if (q) {
+        if (!nvf4 || !q->global || !q->sf) return BSP_ERR_INVALID_ARG;
+        if (N % 64 != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
+        if (!aligned16(q->sf) || (reinterpret_cast<uintptr_t>(q->global) & 3u))
+            return BSP_ERR_MISALIGNED;
+    }
     if (nvf4) {
         if (!sfa || !sfb) return BSP_ERR_INVALID_ARG;
         if (K < 64 || K % 64 != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
@@ -1038,7 +1096,11 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     args.status = device_status_ptr(dev);
     args.wait_ns = wait_ns_override ? wait_ns_override : wait_limit_ns();
     args.debug_stop_iter = debug_stop_iter;
+    args.q_global = q ? q->global : nullptr;
+    args.q_codes = q ? q->codes : nullptr;
+    args.q_sf = q ? q->sf : nullptr;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (q) return launch_pair<true, true>(a, w, args, dev, sms, s, pdl);   // pair kernel only
     const int choice = kernel_choice();
     // the FP8 pair kernel loads whole 128-byte K-atoms (3-D boxes): K % 128 == 0
     const bool pair_ok = nvf4 || K % kBKB == 0;
@@ -1055,15 +1117,6 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
 
 }  // namespace
 
-int nvfp4_gemm_dependent(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
-                         const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
-                         const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
-                         bsp_stream_t stream)
-{
-    return gemm_entry(true, a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias_bf16,
-                      out_bf16, M, N, K, stream, -1, 0, true);
-}
-
 }  // namespace bsp
 
 extern "C" {
@@ -1074,7 +1127,17 @@ int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_globa
                bsp_stream_t stream)
 {
     return bsp::gemm_entry(true, a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias_bf16,
-                           out_bf16, M, N, K, stream, -1, 0, false);
+                           out_bf16, M, N, K, stream, -1, 0);
+}
+
+int nvfp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                     const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                     const void* bias_bf16, const float* out_global, uint8_t* out_codes,
+                     uint8_t* out_sf, int64_t M, int64_t N, int64_t K, bsp_stream_t stream)
+{
+    const bsp::QOut q{out_global, out_codes, out_sf};
+    return bsp::gemm_entry(true, a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias_bf16,
+                           nullptr, M, N, K, stream, -1, 0, &q);
 }
 
 int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_e4m3,
@@ -1082,7 +1145,7 @@ int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_
               int64_t N, int64_t K, bsp_stream_t stream)
 {
     return bsp::gemm_entry(false, a_e4m3, nullptr, a_row_scale, w_e4m3, nullptr, w_row_scale,
-                           bias_bf16, out_bf16, M, N, K, stream, -1, 0, false);
+                           bias_bf16, out_bf16, M, N, K, stream, -1, 0);
 }
 
 int bsp_testing_set_gemm_kernel(int choice)
@@ -1103,7 +1166,7 @@ int bsp_testing_gemm_stall(int scheme, const uint8_t* a, const uint8_t* a_sf, co
     if (scheme != 0 && scheme != 1) return BSP_ERR_INVALID_ARG;
     return bsp::gemm_entry(scheme == 1, a, a_sf, a_scale, w, w_sf, w_scale, nullptr, out_bf16, M,
                            N, K, stream, stop_after_stages,
-                           static_cast<uint64_t>(wait_limit_ms) * 1000000ull, false);
+                           static_cast<uint64_t>(wait_limit_ms) * 1000000ull);
 }
 
 }  // extern "C"

@@ -49,8 +49,9 @@ int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_
     uint8_t* a_sf = a_codes + bsp::scales_offset(M, K);
     int st = nvfp4_quantize_act(x_bf16, M, K, input_scale, a_codes, a_sf, BSP_SF_MMA, stream);
     if (st != BSP_OK) return st;
-    return bsp::nvfp4_gemm_dependent(a_codes, a_sf, input_scale, w_codes, w_sf, w_scale,
-                                     bias_bf16, out_bf16, M, N, K, stream);
+    // launched as a programmatic dependent of the quantizer (as every GEMM launch is)
+    return nvfp4_gemm(a_codes, a_sf, input_scale, w_codes, w_sf, w_scale, bias_bf16, out_bf16,
+                      M, N, K, stream);
 }
 
 }  // extern "C"

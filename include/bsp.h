@@ -103,11 +103,34 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
  *   acc = sum_k e2m1(a)*e4m3(sa) * e2m1(w)*e4m3(sw), accumulated in fp32 on the
  *   tensor cores.
  * Constraints: K % 64 == 0, K >= 64; N % 8 == 0.  Any M >= 0.
+ * Launch: with programmatic stream serialisation (also fp8r_gemm and nvfp4_gemm_quant).
+ * The kernel reads its inputs and writes its output only after the preceding grid on
+ * the stream has completed, so this is safe after any kernel; after the library's own
+ * quantizer, which triggers early, the GEMM's prologue overlaps the quantizer's tail.
  */
 int nvfp4_gemm(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
                const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
                const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
                bsp_stream_t stream);
+
+/*
+ * nvfp4_gemm_quant -- nvfp4_gemm whose output is handed straight to the next nvfp4
+ * linear: instead of writing Y in bf16, the epilogue quantizes bf16(Y) exactly as
+ * nvfp4_quantize_act would (same block-16 arithmetic, global scale out_global) and
+ * writes the codes and MMA-layout scales ("BFL (fp8r / nvfp4)", Kernels table: every
+ * nvfp4 linear quantizes its activations; in an MLP the second linear's activations
+ * are the first one's output).  Bit-identical to nvfp4_gemm followed by
+ * nvfp4_quantize_act(Y, out_global, BSP_SF_MMA), without the bf16 round trip.
+ *   out_global  device fp32: the next layer's input_scale.
+ *   out_codes   [M][N/2] bytes, packed E2M1 ; out_sf  nvfp4_sf_bytes(M, N, BSP_SF_MMA)
+ *               bytes (padding rows of the last 128-row tile are not written).
+ * Other arguments as nvfp4_gemm.  Constraints: those of nvfp4_gemm and N % 64 == 0.
+ * Always runs the CTA-pair kernel.
+ */
+int nvfp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_sf, const float* a_global,
+                     const uint8_t* w_codes, const uint8_t* w_sf, const float* w_global,
+                     const void* bias_bf16, const float* out_global, uint8_t* out_codes,
+                     uint8_t* out_sf, int64_t M, int64_t N, int64_t K, bsp_stream_t stream);
 
 /*
  * nvfp4_linear -- the nvfp4 linear forward in one call ("BFL (fp8r / nvfp4)", Kernels

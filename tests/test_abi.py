@@ -130,6 +130,18 @@ def test_noalloc_size_limit_on_host():
     assert L.nvfp4_linear_noalloc(P, P, P, P, P, None, P, 0, 128, 256, None) == OK
 
 
+def test_gemm_quant_validation_on_host():
+    L = bsp.lib()
+    gq = L.nvfp4_gemm_quant
+    assert gq(P, P, P, P, P, P, None, None, P, P, 128, 128, 256, None) == INVALID   # no out_global
+    assert gq(P, P, P, P, P, P, None, P, P, None, 128, 128, 256, None) == INVALID   # no out_sf
+    assert gq(P, P, P, P, P, P, None, P, None, P, 128, 128, 256, None) == INVALID   # no codes
+    assert gq(P, P, P, P, P, P, None, P, P, P, 128, 96, 256, None) == SHAPE         # N % 64
+    assert gq(P, P, P, P, P, P, None, P, P, P + 8, 128, 128, 256, None) == MISALIGNED
+    assert gq(P, P, P, P, P, P, None, P + 2, P, P, 128, 128, 256, None) == MISALIGNED
+    assert gq(P, P, P, P, P, P, None, P, P, P, 0, 128, 256, None) == OK             # empty
+
+
 def test_testing_hook_validation():
     L = bsp.lib()
     h = L.bsp_testing_gemm_stall
