@@ -54,6 +54,9 @@ def parse():
     p.add_argument("--m", type=int, default=0,
                    help="token count (rows of A) instead of the workload's own, e.g. the fp8r "
                         "sweep 256 / 1024 / 16384")
+    p.add_argument("--dynamic", action="store_true",
+                   help="NVFP4: compute the activation global scale from each step's input "
+                        "(nvfp4_linear_dynamic) instead of the calibrated constant")
     p.add_argument("--chain", nargs="?", const="fused", default=None,
                    choices=["fused", "unfused"],
                    help="MLP workloads: time the up projection, the re-quantization of its output "
@@ -268,6 +271,12 @@ def run_bsp(args):
             ac, asf, ga, wc, wsf, gw, bias=bias, out=y), "TFLOP/s", flops, mm_peak))
         # the whole path in one call: quantizer, then the GEMM as its programmatic dependent
         step_fns = [lambda: bsp.nvfp4_linear(A, ga, wc, wsf, gw, bias=bias, out=y, workspace=ws)]
+        if args.dynamic:
+            gdyn = torch.empty((1,), dtype=torch.float32, device=dev)
+            parts.insert(0, ("nvfp4_global_scale (dynamic)", lambda: bsp.nvfp4_global_scale(
+                A, out=gdyn), "GB/s", M * K * 2.0, hbm))
+            step_fns = [lambda: bsp.nvfp4_linear_dynamic(A, wc, wsf, gw, bias=bias, out=y,
+                                                         input_scale_out=gdyn, workspace=ws)]
         y_out = y
         if args.chain:
             # MLP down projection on GEMM1's output: a6 re-quantizes it with a scale
@@ -403,11 +412,13 @@ def run_bsp(args):
         rate = work / (ms * 1e-3) / (1e9 if unit == "GB/s" else 1e12)
         kernels[name] = {"us": 1e3 * ms, unit: rate, "frac_peak": rate / peak, "peak": peak,
                          "work_per_launch": work}
-    gname, _, _, _, _ = parts[1]
+    gname = next(p[0] for p in parts if p[2] == "TFLOP/s")
     gemm_tflops = kernels[gname]["TFLOP/s"]
     if nvf4:
         step_desc = ("nvfp4_linear = nvfp4_quantize_act + nvfp4_gemm (fused alpha, bias, bf16; "
                      "GEMM as programmatic dependent)")
+        if args.dynamic:
+            step_desc = "nvfp4_linear_dynamic = nvfp4_global_scale of the step's input + " + step_desc
         if args.chain == "fused":
             step_desc = ("nvfp4_quantize_act + nvfp4_gemm_quant (up projection, its output "
                          "re-quantized in the epilogue) + nvfp4_gemm (down projection), each "

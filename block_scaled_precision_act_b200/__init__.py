@@ -21,7 +21,7 @@ import torch
 __all__ = [
     "BSPError", "SF_LINEAR", "SF_MMA", "lib", "library_path",
     "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_quant", "fp8r_quantize_rows", "fp8r_gemm",
-    "nvfp4_linear", "nvfp4_linear_workspace_bytes", "nvfp4_linear_noalloc",
+    "nvfp4_linear", "nvfp4_linear_dynamic", "nvfp4_linear_workspace_bytes", "nvfp4_linear_noalloc",
     "nvfp4_linear_noalloc_max_bytes",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
@@ -47,6 +47,8 @@ _SIGS = {
     "nvfp4_linear": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64,
                       _c_vp, _c_i64, _c_vp], _c_int),
     "nvfp4_linear_workspace_bytes": ([_c_i64, _c_i64], _c_i64),
+    "nvfp4_linear_dynamic": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
+                              _c_i64, _c_vp, _c_i64, _c_vp], _c_int),
     "nvfp4_linear_noalloc": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64,
                               _c_i64, _c_vp], _c_int),
     "nvfp4_linear_noalloc_max_bytes": ([], _c_i64),
@@ -242,6 +244,29 @@ def nvfp4_linear_noalloc(x: torch.Tensor, input_scale: torch.Tensor, w_codes, w_
                                       _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K,
                                       _stream(stream)))
     return out
+
+
+def nvfp4_linear_dynamic(x: torch.Tensor, w_codes, w_sf, w_scale, bias=None, out=None,
+                         input_scale_out=None, workspace=None, stream=None):
+    """nvfp4_linear with input_scale = amax(x) / (448*6) computed on the device for this
+    call; returns (out, input_scale_out)."""
+    _dtype(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = w_codes.shape[0]
+    if w_codes.shape[1] * 2 != K:
+        raise BSPError("nvfp4_linear_dynamic (K mismatch)", -1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if input_scale_out is None:
+        input_scale_out = torch.empty((1,), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((max(nvfp4_linear_workspace_bytes(M, K), 0),), dtype=torch.uint8,
+                                device=x.device)
+    _check("nvfp4_linear_dynamic",
+           lib().nvfp4_linear_dynamic(_ptr(x), _ptr(input_scale_out), _ptr(w_codes), _ptr(w_sf),
+                                      _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K,
+                                      _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out, input_scale_out
 
 
 def fp8r_quantize_rows(x: torch.Tensor, q=None, row_scale=None, stream=None):

@@ -54,4 +54,23 @@ int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_
                       M, N, K, stream);
 }
 
+int nvfp4_linear_dynamic(const void* x_bf16, float* input_scale_out, const uint8_t* w_codes,
+                         const uint8_t* w_sf, const float* w_scale, const void* bias_bf16,
+                         void* out_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                         int64_t workspace_bytes, bsp_stream_t stream)
+{
+    if (M < 0 || N < 0 || K <= 0) return BSP_ERR_INVALID_ARG;
+    if (K % 64 != 0) return BSP_ERR_UNSUPPORTED_SHAPE;
+    if (M == 0 || N == 0) return BSP_OK;
+    if (!input_scale_out) return BSP_ERR_INVALID_ARG;
+    const int64_t need = nvfp4_linear_workspace_bytes(M, K);
+    if (need < 0) return static_cast<int>(need);
+    if (!workspace || workspace_bytes < need) return BSP_ERR_INVALID_ARG;
+    // g = amax(x) / (448 * 6) of this very activation, then the static-scale path with it
+    int st = nvfp4_global_scale(x_bf16, M * K, input_scale_out, stream);
+    if (st != BSP_OK) return st;
+    return nvfp4_linear(x_bf16, input_scale_out, w_codes, w_sf, w_scale, bias_bf16, out_bf16, M,
+                        N, K, workspace, workspace_bytes, stream);
+}
+
 }  // extern "C"

@@ -160,6 +160,21 @@ int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_
                  void* out_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
                  int64_t workspace_bytes, bsp_stream_t stream);
 
+/*
+ * nvfp4_linear_dynamic -- nvfp4_linear with the activation global scale computed from
+ * this call's activations instead of a calibrated constant ("BFL (fp8r / nvfp4)",
+ * nvfp4 bullet: `input_scale` is an fp32 activation scale; here g = amax(x) / (448*6),
+ * the global-scale convention used for the weights): nvfp4_global_scale(x) into
+ * *input_scale_out, then nvfp4_linear with it.  input_scale_out is a device fp32 the
+ * caller owns; it holds g when the call's work completes.  Other arguments, workspace
+ * rules and errors as nvfp4_linear.  Costs one more read of x (an atomic-max pass) than
+ * nvfp4_linear.
+ */
+int nvfp4_linear_dynamic(const void* x_bf16, float* input_scale_out, const uint8_t* w_codes,
+                         const uint8_t* w_sf, const float* w_scale, const void* bias_bf16,
+                         void* out_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
+                         int64_t workspace_bytes, bsp_stream_t stream);
+
 /* Workspace bytes nvfp4_linear needs for an [M][K] activation (codes, padding to 256
  * bytes, MMA-layout scales); negative on bad arguments. */
 int64_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K);

@@ -142,6 +142,16 @@ def test_gemm_quant_validation_on_host():
     assert gq(P, P, P, P, P, P, None, P, P, P, 0, 128, 256, None) == OK             # empty
 
 
+def test_linear_dynamic_validation_on_host():
+    L = bsp.lib()
+    d = L.nvfp4_linear_dynamic
+    need = bsp.nvfp4_linear_workspace_bytes(128, 256)
+    assert d(P, None, P, P, P, None, P, 128, 128, 256, P, need, None) == INVALID   # no g out
+    assert d(P, P, P, P, P, None, P, 128, 128, 256, P, need - 1, None) == INVALID
+    assert d(P, P, P, P, P, None, P, 128, 128, 96, P, need, None) == SHAPE
+    assert d(P, P, P, P, P, None, P, 0, 128, 256, None, 0, None) == OK
+
+
 def test_testing_hook_validation():
     L = bsp.lib()
     h = L.bsp_testing_gemm_stall

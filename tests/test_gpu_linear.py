@@ -110,3 +110,23 @@ def test_linear_rejects_small_workspace():
                      device="cuda")
     with pytest.raises(bsp.BSPError):
         bsp.nvfp4_linear(a, g, w, sf, g, workspace=ws)
+
+
+def test_linear_dynamic_scale():
+    """The dynamic variant: g = amax(x)/2688 of this call's x (the oracle's value, bit
+    for bit), and the output of nvfp4_linear with that g."""
+    M, N, K = 300, 512, 1024
+    a_cpu = synth.bf16_normal((M, K), 1.0, 400, 0.01, 20.0)
+    a = a_cpu.cuda()
+    w = synth.bf16_normal((N, K), 0.02, 401).cuda()
+    wc, wsf, gw = prepared_weight(w)
+    y, g = bsp.nvfp4_linear_dynamic(a, wc, wsf, gw)
+    ref = bsp.nvfp4_linear(a, bsp.nvfp4_global_scale(a), wc, wsf, gw)
+    torch.cuda.synchronize()
+    assert bsp.bsp_last_device_status() == 0
+    assert g.item() == float(oracle.nvfp4_global_scale(a_cpu))
+    assert torch.equal(y, ref)
+    # a second call on a scaled input recomputes g
+    y2, g2 = bsp.nvfp4_linear_dynamic(a * 4, wc, wsf, gw)
+    torch.cuda.synchronize()
+    assert g2.item() == 4 * g.item()
