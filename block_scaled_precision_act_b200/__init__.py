@@ -25,7 +25,7 @@ __all__ = [
     "nvfp4_linear_noalloc_max_bytes",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
-    "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel",
+    "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel", "bsp_testing_set_quant_kernel",
 ]
 
 SF_LINEAR = 0
@@ -63,6 +63,7 @@ _SIGS = {
     "bsp_status_string": ([_c_int], ctypes.c_char_p),
     "bsp_version": ([], _c_int),
     "bsp_testing_set_gemm_kernel": ([_c_int], _c_int),
+    "bsp_testing_set_quant_kernel": ([_c_int], _c_int),
     "bsp_testing_gemm_stall": ([_c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64,
                                 _c_i64, _c_i64, _c_i64, _c_i64, _c_vp], _c_int),
 }
@@ -348,4 +349,12 @@ def bsp_testing_set_gemm_kernel(choice: int) -> int:
     old = int(lib().bsp_testing_set_gemm_kernel(choice))
     if old < 0:
         raise BSPError("bsp_testing_set_gemm_kernel", old)
+    return old
+
+
+def bsp_testing_set_quant_kernel(choice: int) -> int:
+    """Test hook: 0 = by size, 1 = grid-stride quantizer kernel, 2 = staged kernel."""
+    old = int(lib().bsp_testing_set_quant_kernel(choice))
+    if old < 0:
+        raise BSPError("bsp_testing_set_quant_kernel", old)
     return old

@@ -104,6 +104,14 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
     }
 }
 
+// Wait that ignores the abort flag (used on the way out, to drain work in flight).
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
+                                           int* status)
+{
+    volatile int never = 0;
+    return mbar_wait(bar, parity, &never, limit_ns, status, 90);
+}
+
 // ----------------------------------------------------------------- programmatic dependent launch
 // Block until every grid this one depends on (a launch with programmatic stream
 // serialisation) has completed and its memory writes are visible; a no-op for a

@@ -86,14 +86,6 @@ struct Cfg {
     static_assert(BN % 128 == 0 && BN <= 256, "tile width");
 };
 
-// Wait that ignores the abort flag (used on the way out, to drain work in flight).
-__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns,
-                                           int* status)
-{
-    volatile int never = 0;
-    return mbar_wait(bar, parity, &never, limit_ns, status, 90);
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);

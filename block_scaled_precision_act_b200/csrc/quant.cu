@@ -13,10 +13,13 @@
 //   nvfp4: t = 6g ; s = t > 0 ? amax/t : 0 ; sb = E4M3(s) ; d = dec(sb)*g ;
 //          d == 0 -> codes 0 ; else code = E2M1(x * min(1/d, FLT_MAX))
 //   fp8r : s = amax/448 ; s == 0 -> codes 0 ; else q = E4M3(x * min(1/s, FLT_MAX))
+#include <atomic>
 #include <cfloat>
 #include <cstdint>
+#include <mutex>
 
 #include "bsp_internal.h"
+#include "bsp_testing.h"
 #include "bsp_ptx.cuh"
 #include "nvfp4_block.cuh"
 
@@ -165,6 +168,111 @@ __global__ void __launch_bounds__(kQuantThreads)
     }
 }
 
+// Staged variant: one persistent CTA per SM streams a contiguous range of blocks through
+// a ring of shared-memory chunks filled by bulk asynchronous copies (one thread issues
+// them), so a whole chunk (62 KB) per stage is in flight instead of 64 bytes per thread;
+// 31 consumer warps encode from shared memory exactly as above (same lane <-> block map,
+// same stores).  All waits are bounded.
+constexpr int kStageThreads = 1024;
+constexpr int kStageWarps = kStageThreads / 32 - 1;              // consumer warps
+constexpr int kChunkBlocks = kStageWarps * kQBlocksPerWarp;      // 1984 blocks
+constexpr int kChunkBytes = kChunkBlocks * 32;                   // 62 KB of bf16
+constexpr int kStageRing = 3;
+constexpr int kStageSmem = kStageRing * kChunkBytes + 2 * kStageRing * 8 + 128;
+
+__device__ __forceinline__ uint4 lds128(const uint8_t* p)
+{
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(smem_u32(p)));
+    return v;
+}
+
+template <int LAYOUT, bool IDX32>
+__global__ void __launch_bounds__(kStageThreads, 1)
+    nvfp4_quant_staged_kernel(const uint8_t* __restrict__ x, int64_t nblk, int64_t nb_row,
+                              RowDiv rd, const float* __restrict__ gptr, uint2* __restrict__ codes,
+                              uint8_t* __restrict__ scales, int64_t blocks_per_cta, int* status,
+                              uint64_t wait_ns)
+{
+    // a GEMM launched as this grid's programmatic dependent may start its prologue now;
+    // it still waits for this grid to complete before reading the codes
+    griddep_launch_dependents();
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
+                                               ~uintptr_t(127));
+    uint64_t* full = reinterpret_cast<uint64_t*>(ring + kStageRing * kChunkBytes);
+    uint64_t* empty = full + kStageRing;
+    __shared__ int abort_word;
+    volatile int* abort_flag = &abort_word;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kStageRing; ++i) {
+            mbar_init(full + i, 1);
+            mbar_init(empty + i, kStageWarps);
+        }
+        abort_word = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    const int64_t b0 = static_cast<int64_t>(blockIdx.x) * blocks_per_cta;
+    const int64_t b1 = b0 + blocks_per_cta < nblk ? b0 + blocks_per_cta : nblk;
+    const int64_t nchunks = b1 > b0 ? (b1 - b0 + kChunkBlocks - 1) / kChunkBlocks : 0;
+    if (warp == 0) {
+        if (lane == 0) {
+            int64_t i = 0;
+            for (; i < nchunks; ++i) {
+                const int st = static_cast<int>(i % kStageRing);
+                const uint32_t ph = static_cast<uint32_t>((i / kStageRing) & 1);
+                if (i >= kStageRing &&
+                    !mbar_wait(empty + st, ph ^ 1u, abort_flag, wait_ns, status, 31))
+                    break;
+                const int64_t c = b0 + i * kChunkBlocks;
+                const int64_t nb = b1 - c < kChunkBlocks ? b1 - c : kChunkBlocks;
+                const uint32_t bytes = static_cast<uint32_t>(nb * 32);
+                mbar_arrive_expect_tx(full + st, bytes);
+                bulk_load(ring + st * kChunkBytes, x + c * 32, bytes, full + st);
+            }
+            // every copy into the ring lands before the CTA may exit (abort path)
+            for (int64_t j = (i > kStageRing ? i - kStageRing : 0); j < i; ++j)
+                drain_wait(full + (j % kStageRing), static_cast<uint32_t>((j / kStageRing) & 1),
+                           wait_ns, status);
+        }
+    } else {
+        const float g = __ldg(gptr);
+        const float t = __fmul_rn(6.0f, g);
+        const int64_t kb4 = (nb_row + 3) >> 2;
+        const int cw = warp - 1;
+        for (int64_t i = 0; i < nchunks; ++i) {
+            const int st = static_cast<int>(i % kStageRing);
+            const uint32_t ph = static_cast<uint32_t>((i / kStageRing) & 1);
+            const bool ok = mbar_wait(full + st, ph, abort_flag, wait_ns, status, 32);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            const int64_t c = b0 + i * kChunkBlocks;
+            const int64_t lim = b1 - c < kChunkBlocks ? b1 : c + kChunkBlocks;   // chunk end
+            const uint8_t* src = ring + st * kChunkBytes + cw * kQBlocksPerWarp * 32;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int64_t blk = c + cw * kQBlocksPerWarp + h * 32 + lane;
+                Block16 b;
+                if (blk < lim) {
+                    b.lo = lds128(src + (h * 32 + lane) * 32);
+                    b.hi = lds128(src + (h * 32 + lane) * 32 + 16);
+                } else {
+                    b.lo = make_uint4(0, 0, 0, 0);
+                    b.hi = b.lo;
+                }
+                uint32_t sb;
+                const uint2 w = encode_block(b, g, t, sb);
+                store_block<LAYOUT>(codes, scales, blk, lim, nb_row, kb4, w, sb, lane, rd, IDX32);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty + st);
+        }
+    }
+}
+
 // ---------------------------------------------------------------- fp8r
 constexpr int kRowThreads = 128;
 
@@ -307,6 +415,11 @@ __global__ void sf_to_linear_kernel(const uint8_t* __restrict__ src, uint8_t* __
     }
 }
 
+// NVFP4 quantizer kernel choice: 0 = by size, 1 = grid-stride, 2 = staged (test hook)
+std::atomic<int> g_quant_choice{0};
+
+int quant_kernel_choice() { return g_quant_choice.load(); }
+
 int grid_for(int64_t work_items, int per_block, int num_sms, int blocks_per_sm)
 {
     int64_t need = (work_items + per_block - 1) / per_block;
@@ -336,25 +449,71 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
     int st = check_device(&dev, &sms);
     if (st != BSP_OK) return st;
     const int64_t nblk = M * (K / 16);
-    // at most the resident grid (4 CTAs of 256 threads per SM at 64 registers)
-    const int grid = grid_for(nblk, (kQuantThreads / 32) * kQBlocksPerWarp, sms, 4);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const auto* xv = static_cast<const uint4*>(x_bf16);
-    auto* cv = reinterpret_cast<uint2*>(codes);
-    // 32-bit block indices (row by multiply-high) whenever a warp span past the end still
-    // fits; the linear layout needs no row at all
-    const bool idx32 = nblk + static_cast<int64_t>(grid) * kQuantThreads * 2 < (int64_t{1} << 31);
     const RowDiv rd = row_div(static_cast<uint32_t>(K / 16));
+    const int choice = quant_kernel_choice();
+    // Large inputs: the staged kernel (bulk copies into a shared-memory ring, 85 % of HBM at
+    // 65536 x 3072); below ~96 M elements the grid-stride kernel finishes sooner (its CTAs
+    // start encoding after one 64-byte load instead of a 62 KB chunk).
+    const bool staged = choice == 2 || (choice == 0 && nblk * 16 >= (int64_t{96} << 20));
+    if (!staged) {
+        // at most the resident grid (4 CTAs of 256 threads per SM at 64 registers)
+        const int grid = grid_for(nblk, (kQuantThreads / 32) * kQBlocksPerWarp, sms, 4);
+        const auto* xv = static_cast<const uint4*>(x_bf16);
+        auto* cv = reinterpret_cast<uint2*>(codes);
+        // 32-bit block indices (row by multiply-high) whenever a warp span past the end
+        // still fits; the linear layout needs no row at all
+        const bool idx32 =
+            nblk + static_cast<int64_t>(grid) * kQuantThreads * 2 < (int64_t{1} << 31);
+        if (layout == BSP_SF_LINEAR)
+            nvfp4_quant_kernel<BSP_SF_LINEAR, false><<<grid, kQuantThreads, 0, s>>>(
+                xv, nblk, K / 16, rd, global_scale, cv, scales);
+        else if (idx32)
+            nvfp4_quant_kernel<BSP_SF_MMA, true><<<grid, kQuantThreads, 0, s>>>(
+                xv, nblk, K / 16, rd, global_scale, cv, scales);
+        else
+            nvfp4_quant_kernel<BSP_SF_MMA, false><<<grid, kQuantThreads, 0, s>>>(
+                xv, nblk, K / 16, rd, global_scale, cv, scales);
+        return launch_status();
+    }
+    // one persistent CTA per SM, each a contiguous range of whole 64-block warp spans
+    static std::once_flag attr_once[64];
+    static cudaError_t attr_err[64];
+    std::call_once(attr_once[dev], [dev] {
+        cudaError_t e = cudaSuccess;
+        for (auto k : {nvfp4_quant_staged_kernel<BSP_SF_LINEAR, false>,
+                       nvfp4_quant_staged_kernel<BSP_SF_MMA, true>,
+                       nvfp4_quant_staged_kernel<BSP_SF_MMA, false>})
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageSmem);
+        attr_err[dev] = e;
+    });
+    if (attr_err[dev] != cudaSuccess) return BSP_ERR_CUDA;
+    const int64_t spans = (nblk + kQBlocksPerWarp - 1) / kQBlocksPerWarp;
+    const int64_t spans_per_cta = (spans + sms - 1) / sms;
+    const int64_t bpc = spans_per_cta * kQBlocksPerWarp;
+    const int grid = static_cast<int>((nblk + bpc - 1) / bpc);
+    const auto* xb = static_cast<const uint8_t*>(x_bf16);
+    auto* cv = reinterpret_cast<uint2*>(codes);
+    const bool idx32 = nblk < (int64_t{1} << 31) - kChunkBlocks;
+    int* status = device_status_ptr(dev);
+    const uint64_t wns = wait_limit_ns();
     if (layout == BSP_SF_LINEAR)
-        nvfp4_quant_kernel<BSP_SF_LINEAR, false><<<grid, kQuantThreads, 0, s>>>(
-            xv, nblk, K / 16, rd, global_scale, cv, scales);
+        nvfp4_quant_staged_kernel<BSP_SF_LINEAR, false><<<grid, kStageThreads, kStageSmem, s>>>(
+            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
     else if (idx32)
-        nvfp4_quant_kernel<BSP_SF_MMA, true><<<grid, kQuantThreads, 0, s>>>(
-            xv, nblk, K / 16, rd, global_scale, cv, scales);
+        nvfp4_quant_staged_kernel<BSP_SF_MMA, true><<<grid, kStageThreads, kStageSmem, s>>>(
+            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
     else
-        nvfp4_quant_kernel<BSP_SF_MMA, false><<<grid, kQuantThreads, 0, s>>>(
-            xv, nblk, K / 16, rd, global_scale, cv, scales);
+        nvfp4_quant_staged_kernel<BSP_SF_MMA, false><<<grid, kStageThreads, kStageSmem, s>>>(
+            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
     return launch_status();
+}
+
+int bsp_testing_set_quant_kernel(int choice)
+{
+    if (choice < 0 || choice > 2) return BSP_ERR_INVALID_ARG;
+    return bsp::g_quant_choice.exchange(choice);
 }
 
 int fp8r_quantize_rows(const void* x_bf16, int64_t M, int64_t K, uint8_t* q_e4m3,

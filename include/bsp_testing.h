@@ -40,6 +40,16 @@ int bsp_testing_gemm_stall(int scheme, const uint8_t* a, const uint8_t* a_sf,
  */
 int bsp_testing_set_gemm_kernel(int choice);
 
+/*
+ * bsp_testing_set_quant_kernel -- selects the kernel of later nvfp4_quantize_act calls in
+ * this process: 0 = by input size (default), 1 = grid-stride kernel (each thread loads its
+ * blocks directly), 2 = staged kernel (one CTA per SM streaming its range through a
+ * shared-memory ring filled by bulk copies).  Both give identical codes and scales; this
+ * exists so the tests can cover each.  Returns the previous choice, or
+ * BSP_ERR_INVALID_ARG.
+ */
+int bsp_testing_set_quant_kernel(int choice);
+
 #ifdef __cplusplus
 }
 #endif

@@ -158,6 +158,8 @@ def test_testing_hook_validation():
     assert h(1, P, P, P, P, P, P, P, 128, 128, 256, -1, 100, None) == INVALID
     assert h(1, P, P, P, P, P, P, P, 128, 128, 256, 1, 0, None) == INVALID
     assert h(7, P, P, P, P, P, P, P, 128, 128, 256, 1, 100, None) == INVALID
+    assert L.bsp_testing_set_quant_kernel(7) == INVALID
+    assert bsp.bsp_testing_set_quant_kernel(0) == 0
 
 
 def test_python_binding_refuses_cpu_tensors():

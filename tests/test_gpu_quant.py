@@ -13,6 +13,16 @@ from parity import sf_valid_mask
 pytestmark = pytest.mark.gpu
 
 
+@pytest.fixture(params=["grid", "staged"], autouse=True)
+def quant_kernel(request):
+    """Run every quantizer test on both NVFP4 quantizer kernels: the grid-stride one and
+    the staged one (bulk copies into a shared-memory ring); the size-based default picks
+    the staged kernel only for inputs of 96 M elements and more."""
+    old = bsp.bsp_testing_set_quant_kernel({"grid": 1, "staged": 2}[request.param])
+    yield request.param
+    bsp.bsp_testing_set_quant_kernel(old)
+
+
 def gpu_quant(x_cpu, g, layout):
     x = x_cpu.cuda()
     gd = torch.tensor([float(g)], dtype=torch.float32, device="cuda")
