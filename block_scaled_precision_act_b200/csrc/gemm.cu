@@ -489,6 +489,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             // it has completed.  Everything else in the kernel follows these loads.
             griddep_wait();
             int64_t it = 0;
+            int s = 0;                       // ring slot and its phase, kept incrementally
+            uint32_t ph = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
                 const int mt = tile % num_m, nt = tile / num_m;
@@ -496,8 +498,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 const int b_row = nt * 256 + static_cast<int>(rank) * 128;
                 for (int kt = 0; kt < num_kt; ++kt) {
                     if (it == args.debug_stop_iter) { ok = false; break; }
-                    const int s = static_cast<int>(it % STAGES);
-                    const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
                     if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.wait_ns, args.status, 11)) {
                         ok = false;
                         break;
@@ -525,6 +525,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         tma_load_3d_pair(sSFB + s * C::SFB_BYTES, &tmSFB, bar0, 0, 4 * kt, nt * 2);
                     }
                     ++it;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
                 }
             }
             if (rank == 0) {
@@ -536,7 +540,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA issuer (CTA 0)
         if (lane == 0 && rank == 0) {
-            int64_t it = 0;
+            int s = 0;                       // ring slot and phase, scale buffer and phase
+            uint32_t ph = 0;
+            int b = 0;
+            uint32_t bph = 0;
             int acc_it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
@@ -547,17 +554,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 tc_fence_after();
                 const uint32_t d_tmem = tbase + static_cast<uint32_t>((acc_it & 1) * C::ACC_STRIDE);
                 for (int kt = 0; kt < num_kt; ++kt) {
-                    const int s = static_cast<int>(it % STAGES);
-                    const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
-                    const int b = static_cast<int>(it & 1);
-                    if (!mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status, 13)) {
+                    // NVFP4: the copy warps hand over a stage's scales only after they have
+                    // seen its `full` barrier complete, so waiting on `sf_full` alone also
+                    // orders the MMAs after the stage's operand loads (one wait per stage).
+                    if (!NVF4 &&
+                        !mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status, 13)) {
                         ok = false;
                         break;
                     }
                     int nk;
                     if constexpr (NVF4) {
-                        if (!mbar_wait(sf_full + b, static_cast<uint32_t>((it >> 1) & 1), abort_flag,
-                                       args.wait_ns, args.status, 15)) {
+                        if (!mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status,
+                                       15)) {
                             ok = false;
                             break;
                         }
@@ -583,7 +591,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     }
                     tc_commit_pair(empty + s, 0x1);
                     if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
-                    ++it;
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                    b ^= 1;
+                    bph ^= static_cast<uint32_t>(b == 0);
                 }
                 if (!ok) break;
                 tc_commit_pair(acc_full, 0x3);
@@ -595,14 +608,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         if constexpr (NVF4) {
             if (lane == 0 && rank == 0) {
                 const int which = warp - 2;          // 0: SFA, 1: SFB rows 0-127, 2: rows 128-255
-                int64_t it = 0;
+                int s = 0;
+                uint32_t ph = 0;
+                int b = 0;
+                uint32_t bph = 0;
                 bool ok = true;
                 for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
                     for (int kt = 0; kt < num_kt; ++kt) {
-                        const int s = static_cast<int>(it % STAGES);
-                        const uint32_t ph = static_cast<uint32_t>((it / STAGES) & 1);
-                        const int b = static_cast<int>(it & 1);
-                        if (!mbar_wait(sf_empty + b, static_cast<uint32_t>(((it >> 1) & 1) ^ 1),
+                        if (!mbar_wait(sf_empty + b, bph ^ 1u,
                                        abort_flag, args.wait_ns, args.status, 16) ||
                             !mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status, 17)) {
                             ok = false;
@@ -622,8 +635,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                                     sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES +
                                                             (which - 1) * 2048 + kb * 512)));
                         }
-                        tc_commit_pair(sf_full + b, 0x1);
-                        ++it;
+                        // Hand the buffer over with a fence and a plain arrive, not a commit:
+                        // the MMAs that read it are issued after this arrive and queue behind
+                        // these copies in the pair's in-order tensor pipe, whereas a commit
+                        // would complete only after the MMAs already queued ahead of it.
+                        tc_fence_before();
+                        mbar_arrive(sf_full + b);
+                        if (++s == STAGES) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                        b ^= 1;
+                        bph ^= static_cast<uint32_t>(b == 0);
                     }
                 }
                 tc_commit_pair(cp_fin, 0x1);     // lets the teardown wait for every copy
