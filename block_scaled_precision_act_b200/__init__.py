@@ -22,7 +22,7 @@ __all__ = [
     "BSPError", "SF_LINEAR", "SF_MMA", "lib", "library_path",
     "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_quant", "fp8r_quantize_rows", "fp8r_gemm",
     "nvfp4_linear", "nvfp4_linear_dynamic", "nvfp4_linear_workspace_bytes", "nvfp4_linear_noalloc",
-    "nvfp4_linear_noalloc_max_bytes",
+    "nvfp4_linear_noalloc_max_bytes", "fp8r_linear", "fp8r_linear_workspace_bytes",
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
     "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel", "bsp_testing_set_quant_kernel",
@@ -53,6 +53,9 @@ _SIGS = {
                               _c_i64, _c_vp], _c_int),
     "nvfp4_linear_noalloc_max_bytes": ([], _c_i64),
     "fp8r_quantize_rows": ([_c_vp, _c_i64, _c_i64, _c_vp, _c_vp, _c_vp], _c_int),
+    "fp8r_linear": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp, _c_i64,
+                     _c_vp], _c_int),
+    "fp8r_linear_workspace_bytes": ([_c_i64, _c_i64], _c_i64),
     "fp8r_gemm": ([_c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64, _c_i64, _c_i64, _c_vp],
                   _c_int),
     "nvfp4_global_scale": ([_c_vp, _c_i64, _c_vp, _c_vp], _c_int),
@@ -281,6 +284,34 @@ def fp8r_quantize_rows(x: torch.Tensor, q=None, row_scale=None, stream=None):
     _check("fp8r_quantize_rows",
            lib().fp8r_quantize_rows(_ptr(x), M, K, _ptr(q), _ptr(row_scale), _stream(stream)))
     return q, row_scale
+
+
+def fp8r_linear_workspace_bytes(M: int, K: int) -> int:
+    n = lib().fp8r_linear_workspace_bytes(M, K)
+    if n < 0:
+        raise BSPError("fp8r_linear_workspace_bytes", int(n))
+    return int(n)
+
+
+def fp8r_linear(x: torch.Tensor, w_q, w_row_scale, bias=None, out=None, workspace=None,
+                stream=None):
+    """Y[M, N] bf16 = fp8r linear of bf16 x [M, K]: row quantizer + FP8 GEMM in one call.
+    `workspace` (uint8, at least fp8r_linear_workspace_bytes(M, K) bytes) is allocated here
+    when not given."""
+    _dtype(x, torch.bfloat16, "x")
+    M, K = x.shape
+    N = w_q.shape[0]
+    if w_q.shape[1] != K:
+        raise BSPError("fp8r_linear (K mismatch)", -1)
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if workspace is None:
+        workspace = torch.empty((max(fp8r_linear_workspace_bytes(M, K), 0),),
+                                dtype=torch.uint8, device=x.device)
+    _check("fp8r_linear",
+           lib().fp8r_linear(_ptr(x), _ptr(w_q), _ptr(w_row_scale), _ptr(bias), _ptr(out), M, N, K,
+                             _ptr(workspace), workspace.numel(), _stream(stream)))
+    return out
 
 
 def fp8r_gemm(a_q, a_row_scale, w_q, w_row_scale, bias=None, out=None, stream=None):

@@ -19,6 +19,8 @@ int64_t scales_offset(int64_t M, int64_t K)
     return (codes_bytes(M, K) + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign;
 }
 
+int64_t align_up(int64_t v) { return (v + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign; }
+
 }  // namespace
 }  // namespace bsp
 
@@ -71,6 +73,31 @@ int nvfp4_linear_dynamic(const void* x_bf16, float* input_scale_out, const uint8
     if (st != BSP_OK) return st;
     return nvfp4_linear(x_bf16, input_scale_out, w_codes, w_sf, w_scale, bias_bf16, out_bf16, M,
                         N, K, workspace, workspace_bytes, stream);
+}
+
+int64_t fp8r_linear_workspace_bytes(int64_t M, int64_t K)
+{
+    if (M < 0 || K <= 0 || K % 8 != 0) return BSP_ERR_INVALID_ARG;
+    if (M > (int64_t{1} << 40) / K) return BSP_ERR_UNSUPPORTED_SHAPE;
+    return bsp::align_up(M * K) + bsp::align_up(4 * M);
+}
+
+int fp8r_linear(const void* x_bf16, const uint8_t* w_e4m3, const float* w_row_scale,
+                const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
+                void* workspace, int64_t workspace_bytes, bsp_stream_t stream)
+{
+    if (M < 0 || N < 0 || K <= 0) return BSP_ERR_INVALID_ARG;
+    if (M == 0 || N == 0) return BSP_OK;
+    const int64_t need = fp8r_linear_workspace_bytes(M, K);
+    if (need < 0) return static_cast<int>(need);
+    if (!workspace || workspace_bytes < need) return BSP_ERR_INVALID_ARG;
+    if (!bsp::aligned16(workspace)) return BSP_ERR_MISALIGNED;
+    auto* aq = static_cast<uint8_t*>(workspace);
+    auto* as = reinterpret_cast<float*>(aq + bsp::align_up(M * K));
+    int st = fp8r_quantize_rows(x_bf16, M, K, aq, as, stream);
+    if (st != BSP_OK) return st;
+    // launched as a programmatic dependent of the quantizer (as every GEMM launch is)
+    return fp8r_gemm(aq, as, w_e4m3, w_row_scale, bias_bf16, out_bf16, M, N, K, stream);
 }
 
 }  // extern "C"

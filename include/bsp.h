@@ -231,6 +231,27 @@ int fp8r_gemm(const uint8_t* a_e4m3, const float* a_row_scale, const uint8_t* w_
               int64_t N, int64_t K, bsp_stream_t stream);
 
 /*
+ * fp8r_linear -- the fp8r linear forward in one call ("BFL (fp8r / nvfp4)", fp8r bullet
+ * and Kernels table: activations quantized to E4M3 per row at run time, then the
+ * row-scaled FP8 GEMM): fp8r_quantize_rows(x) into `workspace`, then fp8r_gemm (launched
+ * as the quantizer's programmatic dependent).  Results are bit-identical to the two calls.
+ *   x_bf16 [M][K] bf16 ; w_e4m3 [N][K] ; w_row_scale [N] fp32 ; bias [N] bf16 or NULL ;
+ *   out_bf16 [M][N].
+ *   workspace  caller-owned device buffer of at least fp8r_linear_workspace_bytes(M, K)
+ *              bytes, 16-byte aligned (codes, then the row scales at a 256-byte boundary);
+ *              fully rewritten by each call; not shared by calls that can run at the same
+ *              time.
+ * Constraints: those of fp8r_quantize_rows and fp8r_gemm.  Errors as those two, and
+ * BSP_ERR_INVALID_ARG for a missing or too small workspace.
+ */
+int fp8r_linear(const void* x_bf16, const uint8_t* w_e4m3, const float* w_row_scale,
+                const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
+                void* workspace, int64_t workspace_bytes, bsp_stream_t stream);
+
+/* Workspace bytes fp8r_linear needs for an [M][K] activation; negative on bad arguments. */
+int64_t fp8r_linear_workspace_bytes(int64_t M, int64_t K);
+
+/*
  * nvfp4_global_scale -- g = amax(X) / (448 * 6) over n bf16 values, written to the
  * device fp32 at `global_scale_out` (the nvfp4 `weight_scale_2` / `input_scale`
  * convention: a decode-side multiplier that maps the largest block scale to the

@@ -152,6 +152,20 @@ def test_linear_dynamic_validation_on_host():
     assert d(P, P, P, P, P, None, P, 0, 128, 256, None, 0, None) == OK
 
 
+def test_fp8r_linear_workspace_and_validation_on_host():
+    L = bsp.lib()
+    a256 = lambda v: (v + 255) // 256 * 256
+    assert bsp.fp8r_linear_workspace_bytes(256, 3072) == a256(256 * 3072) + a256(1024)
+    assert bsp.fp8r_linear_workspace_bytes(4096, 3072) == a256(4096 * 3072) + a256(4 * 4096)
+    assert L.fp8r_linear_workspace_bytes(256, 12) == INVALID
+    f = L.fp8r_linear
+    need = bsp.fp8r_linear_workspace_bytes(128, 256)
+    assert f(P, P, P, None, P, 128, 128, 256, None, need, None) == INVALID
+    assert f(P, P, P, None, P, 128, 128, 256, P, need - 1, None) == INVALID
+    assert f(P, P, P, None, P, 128, 128, 256, P + 8, need, None) == MISALIGNED
+    assert f(P, P, P, None, P, 0, 128, 256, None, 0, None) == OK
+
+
 def test_testing_hook_validation():
     L = bsp.lib()
     h = L.bsp_testing_gemm_stall
