@@ -17,6 +17,14 @@ int* device_status_ptr(int device);
 // Bounded-wait limit for kernels, in nanoseconds.
 uint64_t wait_limit_ns();
 
+// nvfp4_gemm (nvf4) / fp8r_gemm launched right after the library's activation quantizer
+// wrote `a` (and `a_sf`): same results, but the weight operand's first stages are fetched
+// while that quantizer finishes (the quantizer never writes the weights).
+int gemm_after_quantizer(bool nvf4, const uint8_t* a, const uint8_t* a_sf, const float* a_scale,
+                         const uint8_t* w, const uint8_t* w_sf, const float* w_scale,
+                         const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
+                         bsp_stream_t stream);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int launch_status()

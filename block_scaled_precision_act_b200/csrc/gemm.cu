@@ -61,6 +61,10 @@ struct GemmArgs {
     const float* q_global;           // device fp32 global scale g of the next layer
     uint8_t* q_codes;                // [M][N/2] E2M1 codes of bf16(Y)
     uint8_t* q_sf;                   // E4M3 block scales of bf16(Y), MMA layout, K = N
+    // the weight operand (B, its scales) cannot be written by the grid this launch depends
+    // on, so the pair producer may fetch the first stages of it before griddep_wait
+    // (set only where that grid is the library's own activation quantizer)
+    int w_early;
 };
 
 template <bool NVF4, int BN, int STAGES, int NACC>
@@ -484,9 +488,46 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
-            // Under a programmatic launch the operands may still be being written by
-            // the preceding grid (the activation quantizer): nothing is loaded before
-            // it has completed.  Everything else in the kernel follows these loads.
+            // A stage's loads: the activation operand (A codes, A scales) and the weight
+            // operand (B codes, B scales), all completing on the leader's `full` barrier.
+            auto load_a = [&](int st, int kt, int a_row) {
+                const uint32_t bar0 = mapa_shared(smem_u32(full + st), 0);
+                if constexpr (C::ATOMS == 1) {
+                    tma_load_2d_pair(sA + st * C::A_BYTES, &tmA, bar0, kt * kBKB, a_row);
+                } else {
+                    // operands viewed as [atom][row][128 B]: one box = 128 rows x ATOMS atoms
+                    tma_load_3d_pair(sA + st * C::A_BYTES, &tmA, bar0, 0, a_row, C::ATOMS * kt);
+                }
+                // scale arrays as [row tile][512-byte chunk][64 x 8 bytes]: a stage needs
+                // chunks 4kt..4kt+3 of one (A) or two (B) row tiles: one box each
+                if constexpr (NVF4)
+                    tma_load_3d_pair(sSFA + st * C::SFA_BYTES, &tmSFA, bar0, 0, 4 * kt,
+                                     a_row / 128);
+            };
+            auto load_b = [&](int st, int kt, int b_row, int nt) {
+                const uint32_t bar0 = mapa_shared(smem_u32(full + st), 0);
+                if constexpr (C::ATOMS == 1)
+                    tma_load_2d_pair(sB + st * C::B_BYTES, &tmB, bar0, kt * kBKB, b_row);
+                else
+                    tma_load_3d_pair(sB + st * C::B_BYTES, &tmB, bar0, 0, b_row, C::ATOMS * kt);
+                if constexpr (NVF4)
+                    tma_load_3d_pair(sSFB + st * C::SFB_BYTES, &tmSFB, bar0, 0, 4 * kt, nt * 2);
+            };
+            // The weight operand of the first stages may be fetched before the preceding
+            // grid completes (w_early: that grid is the activation quantizer, which does
+            // not write it); the ring slots are fresh, so no empty-wait is needed.
+            int pre = 0;
+            if (args.w_early && pair < num_tiles && args.debug_stop_iter < 0) {
+                const int nt0 = pair / num_m;
+                pre = num_kt < STAGES ? num_kt : STAGES;
+                for (int kt = 0; kt < pre; ++kt) {
+                    if (rank == 0) mbar_arrive_expect_tx(full + kt, 2 * C::STAGE_TX);
+                    load_b(kt, kt, nt0 * 256 + static_cast<int>(rank) * 128, nt0);
+                }
+            }
+            // Under a programmatic launch the activations may still be being written by
+            // the preceding grid (the activation quantizer): none is loaded before it has
+            // completed.  Everything else in the kernel follows these loads.
             griddep_wait();
             int64_t it = 0;
             int s = 0;                       // ring slot and its phase, kept incrementally
@@ -497,6 +538,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 const int a_row = mt * 256 + static_cast<int>(rank) * 128;
                 const int b_row = nt * 256 + static_cast<int>(rank) * 128;
                 for (int kt = 0; kt < num_kt; ++kt) {
+                    if (it < pre) {              // weight half already issued
+                        load_a(s, kt, a_row);
+                        ++it;
+                        if (++s == STAGES) {
+                            s = 0;
+                            ph ^= 1u;
+                        }
+                        continue;
+                    }
                     if (it == args.debug_stop_iter) { ok = false; break; }
                     if (!mbar_wait(empty + s, ph ^ 1u, abort_flag, args.wait_ns, args.status, 11)) {
                         ok = false;
@@ -507,23 +557,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     // stage costs about half the load bandwidth).
                     if (rank == 0 && it >= STAGES)
                         mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(empty + s), 1));
-                    const uint32_t bar0 = mapa_shared(smem_u32(full + s), 0);
                     if (rank == 0) mbar_arrive_expect_tx(full + s, 2 * C::STAGE_TX);
-                    if constexpr (C::ATOMS == 1) {
-                        tma_load_2d_pair(sA + s * C::A_BYTES, &tmA, bar0, kt * kBKB, a_row);
-                        tma_load_2d_pair(sB + s * C::B_BYTES, &tmB, bar0, kt * kBKB, b_row);
-                    } else {
-                        // operands viewed as [atom][row][128 B]: one box = 128 rows x ATOMS atoms
-                        tma_load_3d_pair(sA + s * C::A_BYTES, &tmA, bar0, 0, a_row, C::ATOMS * kt);
-                        tma_load_3d_pair(sB + s * C::B_BYTES, &tmB, bar0, 0, b_row, C::ATOMS * kt);
-                    }
-                    if constexpr (NVF4) {
-                        // scale arrays as [row tile][512-byte chunk][64 x 8 bytes]: a stage
-                        // needs chunks 4kt..4kt+3 of one (A) or two (B) row tiles: one box each
-                        tma_load_3d_pair(sSFA + s * C::SFA_BYTES, &tmSFA, bar0, 0, 4 * kt,
-                                         a_row / 128);
-                        tma_load_3d_pair(sSFB + s * C::SFB_BYTES, &tmSFB, bar0, 0, 4 * kt, nt * 2);
-                    }
+                    load_a(s, kt, a_row);
+                    load_b(s, kt, b_row, nt);
                     ++it;
                     if (++s == STAGES) {
                         s = 0;
@@ -1072,7 +1108,8 @@ struct QOut {
 int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_scale,
                const uint8_t* w, const uint8_t* sfb, const float* w_scale, const void* bias,
                void* out, int64_t M, int64_t N, int64_t K, bsp_stream_t stream,
-               int64_t debug_stop_iter, uint64_t wait_ns_override, const QOut* q = nullptr)
+               int64_t debug_stop_iter, uint64_t wait_ns_override, const QOut* q = nullptr,
+               bool w_early = false)
 {
     const bool pdl = true;
     int st = check_gemm_common(a, w, bias, q ? static_cast<void*>(q->codes) : out, M, N, K);
@@ -1114,6 +1151,7 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     args.q_global = q ? q->global : nullptr;
     args.q_codes = q ? q->codes : nullptr;
     args.q_sf = q ? q->sf : nullptr;
+    args.w_early = w_early ? 1 : 0;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (q) return launch_pair<true, true>(a, w, args, dev, sms, s, pdl);   // pair kernel only
     const int choice = kernel_choice();
@@ -1131,6 +1169,15 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
 }
 
 }  // namespace
+
+int gemm_after_quantizer(bool nvf4, const uint8_t* a, const uint8_t* a_sf, const float* a_scale,
+                         const uint8_t* w, const uint8_t* w_sf, const float* w_scale,
+                         const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
+                         bsp_stream_t stream)
+{
+    return gemm_entry(nvf4, a, a_sf, a_scale, w, w_sf, w_scale, bias_bf16, out_bf16, M, N, K,
+                      stream, -1, 0, nullptr, true);
+}
 
 }  // namespace bsp
 

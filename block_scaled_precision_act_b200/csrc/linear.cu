@@ -51,9 +51,10 @@ int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_
     uint8_t* a_sf = a_codes + bsp::scales_offset(M, K);
     int st = nvfp4_quantize_act(x_bf16, M, K, input_scale, a_codes, a_sf, BSP_SF_MMA, stream);
     if (st != BSP_OK) return st;
-    // launched as a programmatic dependent of the quantizer (as every GEMM launch is)
-    return nvfp4_gemm(a_codes, a_sf, input_scale, w_codes, w_sf, w_scale, bias_bf16, out_bf16,
-                      M, N, K, stream);
+    // launched as a programmatic dependent of the quantizer (as every GEMM launch is),
+    // fetching its first weight stages while the quantizer finishes
+    return bsp::gemm_after_quantizer(true, a_codes, a_sf, input_scale, w_codes, w_sf, w_scale,
+                                     bias_bf16, out_bf16, M, N, K, stream);
 }
 
 int nvfp4_linear_dynamic(const void* x_bf16, float* input_scale_out, const uint8_t* w_codes,
@@ -96,8 +97,10 @@ int fp8r_linear(const void* x_bf16, const uint8_t* w_e4m3, const float* w_row_sc
     auto* as = reinterpret_cast<float*>(aq + bsp::align_up(M * K));
     int st = fp8r_quantize_rows(x_bf16, M, K, aq, as, stream);
     if (st != BSP_OK) return st;
-    // launched as a programmatic dependent of the quantizer (as every GEMM launch is)
-    return fp8r_gemm(aq, as, w_e4m3, w_row_scale, bias_bf16, out_bf16, M, N, K, stream);
+    // launched as a programmatic dependent of the quantizer (as every GEMM launch is),
+    // fetching its first weight stages while the quantizer finishes
+    return bsp::gemm_after_quantizer(false, aq, nullptr, as, w_e4m3, nullptr, w_row_scale,
+                                     bias_bf16, out_bf16, M, N, K, stream);
 }
 
 }  // extern "C"
