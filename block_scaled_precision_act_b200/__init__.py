@@ -26,6 +26,7 @@ __all__ = [
     "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
     "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel", "bsp_testing_set_quant_kernel",
+    "bsp_testing_cvt_range",
 ]
 
 SF_LINEAR = 0
@@ -67,6 +68,7 @@ _SIGS = {
     "bsp_version": ([], _c_int),
     "bsp_testing_set_gemm_kernel": ([_c_int], _c_int),
     "bsp_testing_set_quant_kernel": ([_c_int], _c_int),
+    "bsp_testing_cvt_range": ([_c_int, ctypes.c_uint32, _c_i64, _c_vp, _c_vp], _c_int),
     "bsp_testing_gemm_stall": ([_c_int, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_vp, _c_i64,
                                 _c_i64, _c_i64, _c_i64, _c_i64, _c_vp], _c_int),
 }
@@ -389,3 +391,13 @@ def bsp_testing_set_quant_kernel(choice: int) -> int:
     if old < 0:
         raise BSPError("bsp_testing_set_quant_kernel", old)
     return old
+
+
+def bsp_testing_cvt_range(kind: int, first: int, n: int, out=None, stream=None):
+    """Test hook: the quantizers' E2M1 (kind 0) / E4M3 (kind 1) conversion of the fp32
+    values with bit patterns first .. first+n-1, as uint8 on the current device."""
+    if out is None:
+        out = torch.empty((n,), dtype=torch.uint8, device="cuda")
+    _check("bsp_testing_cvt_range",
+           lib().bsp_testing_cvt_range(kind, first, n, _ptr(out), _stream(stream)))
+    return out

@@ -420,6 +420,19 @@ std::atomic<int> g_quant_choice{0};
 
 int quant_kernel_choice() { return g_quant_choice.load(); }
 
+// Test hook kernel: the quantizers' conversions (cvt.rn.satfinite.e2m1x2.f32 /
+// .e4m3x2.f32, through the same wrappers) applied to every fp32 whose bit pattern lies
+// in [first, first + n).
+__global__ void cvt_range_kernel(int kind, uint32_t first, int64_t n, uint8_t* __restrict__ out)
+{
+    for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float y = __uint_as_float(first + static_cast<uint32_t>(i));
+        out[i] = static_cast<uint8_t>(kind == 0 ? (cvt_e2m1x2(y, 0.0f) & 0xFu)
+                                                : (cvt_e4m3x2(y, 0.0f) & 0xFFu));
+    }
+}
+
 int grid_for(int64_t work_items, int per_block, int num_sms, int blocks_per_sm)
 {
     int64_t need = (work_items + per_block - 1) / per_block;
@@ -507,6 +520,20 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
     else
         nvfp4_quant_staged_kernel<BSP_SF_MMA, false><<<grid, kStageThreads, kStageSmem, s>>>(
             xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
+    return launch_status();
+}
+
+int bsp_testing_cvt_range(int kind, uint32_t first, int64_t n, uint8_t* out, bsp_stream_t stream)
+{
+    using namespace bsp;
+    if ((kind != 0 && kind != 1) || n < 0 || n > (int64_t{1} << 32) - first) return BSP_ERR_INVALID_ARG;
+    if (n == 0) return BSP_OK;
+    if (!out) return BSP_ERR_INVALID_ARG;
+    int dev = 0, sms = 0;
+    int st = check_device(&dev, &sms);
+    if (st != BSP_OK) return st;
+    const int grid = grid_for(n, 256 * 8, sms, 8);
+    cvt_range_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(kind, first, n, out);
     return launch_status();
 }
 

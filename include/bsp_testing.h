@@ -50,6 +50,16 @@ int bsp_testing_set_gemm_kernel(int choice);
  */
 int bsp_testing_set_quant_kernel(int choice);
 
+/*
+ * bsp_testing_cvt_range -- writes out[i] = the quantizers' conversion of the fp32 whose
+ * bit pattern is first + i, for i in [0, n): kind 0 = E2M1 code (cvt.rn.satfinite.e2m1x2,
+ * the low nibble), kind 1 = E4M3 byte (cvt.rn.satfinite.e4m3x2).  first + n <= 2^32.
+ * An exhaustive pin of the conversions walks all 2^32 patterns in ranges.  Returns
+ * BSP_ERR_INVALID_ARG on a bad kind or range.
+ */
+int bsp_testing_cvt_range(int kind, uint32_t first, int64_t n, uint8_t* out,
+                          bsp_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -46,6 +46,9 @@ def lib():
         L.oracle_e4m3_decode.restype = ctypes.c_float
         L.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         L.oracle_e4m3_encode.restype = ctypes.c_uint8
+        L.oracle_encode_range.argtypes = [ctypes.c_int, ctypes.c_uint32, ctypes.c_int64,
+                                          ctypes.c_void_p]
+        L.oracle_encode_range.restype = None
         L.oracle_sf_bytes.argtypes = [_i64, _i64, ctypes.c_int]
         L.oracle_sf_bytes.restype = _i64
         L.oracle_sf_mma_offset.argtypes = [_i64, _i64, _i64]
@@ -110,6 +113,14 @@ def e4m3_decode(code: int) -> float:
 
 def e4m3_encode(y: float) -> int:
     return int(lib().oracle_e4m3_encode(np.float32(y)))
+
+
+def encode_range(kind: int, first: int, n: int) -> np.ndarray:
+    """Codes of the fp32 values with bit patterns first .. first+n-1 (kind 0: E2M1,
+    1: E4M3), the scalar encoders applied one by one."""
+    out = np.empty(n, dtype=np.uint8)
+    lib().oracle_encode_range(kind, first, n, out.ctypes.data)
+    return out
 
 
 # ---------------------------------------------------------------- scale layouts

@@ -167,6 +167,21 @@ int64_t oracle_sf_mma_offset(int64_t r, int64_t c, int64_t K)
 }
 
 /* Copy a linear-layout scale array into the MMA layout; padding bytes are 0. */
+/* The encoders above applied to every fp32 whose bit pattern is first, first+1, ...,
+ * first+n-1 (an exhaustive pin of a converter walks all 2^32 patterns in ranges).
+ * kind 0: E2M1, kind 1: E4M3. */
+void oracle_encode_range(int kind, uint32_t first, int64_t n, uint8_t* out)
+{
+    e4m3_build();                       /* the table once, before the threads read it */
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; ++i) {
+        uint32_t bits = first + (uint32_t)i;
+        float y;
+        memcpy(&y, &bits, sizeof y);
+        out[i] = kind == 0 ? oracle_e2m1_encode(y) : oracle_e4m3_encode(y);
+    }
+}
+
 void oracle_sf_linear_to_mma(const uint8_t* lin, int64_t R, int64_t K, uint8_t* mma)
 {
     memset(mma, 0, (size_t)oracle_sf_bytes(R, K, 1));
@@ -234,6 +249,7 @@ static void nvfp4_quantize_row(const uint16_t* xr, int64_t K, float g,
 void oracle_nvfp4_quantize(const uint16_t* x, int64_t R, int64_t K, float g,
                            uint8_t* codes, uint8_t* sf_lin, int threads)
 {
+    e4m3_build();                       /* the table once, before the threads read it */
 #ifdef _OPENMP
     if (threads < 1) threads = 1;
     #pragma omp parallel for num_threads(threads) schedule(static)
@@ -281,6 +297,7 @@ static void fp8r_quantize_row(const uint16_t* xr, int64_t K, uint8_t* qr, float*
 void oracle_fp8r_quantize(const uint16_t* x, int64_t R, int64_t K, uint8_t* q, float* s,
                           int threads)
 {
+    e4m3_build();                       /* the table once, before the threads read it */
 #ifdef _OPENMP
     if (threads < 1) threads = 1;
     #pragma omp parallel for num_threads(threads) schedule(static)

@@ -173,6 +173,9 @@ def test_testing_hook_validation():
     assert h(1, P, P, P, P, P, P, P, 128, 128, 256, 1, 0, None) == INVALID
     assert h(7, P, P, P, P, P, P, P, 128, 128, 256, 1, 100, None) == INVALID
     assert L.bsp_testing_set_quant_kernel(7) == INVALID
+    assert L.bsp_testing_cvt_range(2, 0, 16, P, None) == INVALID
+    assert L.bsp_testing_cvt_range(0, 0xFFFFFFF0, 32, P, None) == INVALID    # past 2^32
+    assert L.bsp_testing_cvt_range(0, 0, 0, None, None) == OK
     assert bsp.bsp_testing_set_quant_kernel(0) == 0
 
 
