@@ -65,6 +65,9 @@ struct GemmArgs {
     // on, so the pair producer may fetch the first stages of it before griddep_wait
     // (set only where that grid is the library's own activation quantizer)
     int w_early;
+    // pair kernel, NVFP4: the MMA thread issues each stage's scale-factor copies itself,
+    // in order ahead of the stage's MMAs, instead of the copy warps
+    int sf_inline;
 };
 
 template <bool NVF4, int BN, int STAGES, int NACC>
@@ -397,7 +400,11 @@ struct PairCfg {
     static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
     static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
     static constexpr int OFF_EPI = OFF_SFB + STAGES * SFB_BYTES;
-    static constexpr int OFF_BAR = OFF_EPI + EPI_WARPS * 2 * EPI_SLAB;
+    // NVFP4: each epilogue warp's bias columns of the tile (4 subtiles x 32 bf16),
+    // fetched while the tile's MMAs run
+    static constexpr int BIAS_WARP = NVF4 ? 4 * 32 * 2 : 0;
+    static constexpr int OFF_BIAS = OFF_EPI + EPI_WARPS * 2 * EPI_SLAB;
+    static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_WARP;
     static constexpr int NUM_BARS = 2 * STAGES + 4 + 4;
     static constexpr int SMEM_BYTES = 1024 + OFF_BAR + NUM_BARS * 8 + 16;
     static constexpr int ACC_STRIDE = 160;
@@ -600,13 +607,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     }
                     int nk;
                     if constexpr (NVF4) {
-                        if (!mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status,
-                                       15)) {
-                            ok = false;
-                            break;
+                        if (args.sf_inline) {
+                            // the stage's scale copies go into the pair's in-order tensor
+                            // queue just ahead of the MMAs that read them
+                            if (!mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status,
+                                           13)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            nk = min(4, K / 64 - 4 * kt);
+                            const uint32_t sfd = tbase + C::SF_COL0 + b * C::SF_BUF;
+                            for (int kb = 0; kb < nk; ++kb) {
+                                tmem_cp_32x128b_x4_pair(
+                                    sfd + kb * 4,
+                                    sdesc_sf_block(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512)));
+                                tmem_cp_32x128b_x4_pair(
+                                    sfd + 16 + kb * 8,
+                                    sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES + kb * 512)));
+                                tmem_cp_32x128b_x4_pair(
+                                    sfd + 16 + kb * 8 + 4,
+                                    sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES + 2048 +
+                                                            kb * 512)));
+                            }
+                        } else {
+                            if (!mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status,
+                                           15)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            nk = min(4, K / 64 - 4 * kt);
                         }
-                        tc_fence_after();
-                        nk = min(4, K / 64 - 4 * kt);
                     } else {
                         nk = min(4 * C::ATOMS, (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
                     }
@@ -626,7 +658,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                             mma_f8f6f4_pair(d_tmem, adesc + koff, bdesc + koff, C::IDESC, acc);
                     }
                     tc_commit_pair(empty + s, 0x1);
-                    if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
+                    if constexpr (NVF4)
+                        if (!args.sf_inline) tc_commit_pair(sf_empty + b, 0x1);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -642,7 +675,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     } else if (warp <= 4) {
         // ------------------------------------------------------------ scale copies (CTA 0)
         if constexpr (NVF4) {
-            if (lane == 0 && rank == 0) {
+            if (lane == 0 && rank == 0 && !args.sf_inline) {
                 const int which = warp - 2;          // 0: SFA, 1: SFB rows 0-127, 2: rows 128-255
                 int s = 0;
                 uint32_t ph = 0;
@@ -695,32 +728,62 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         const int h = ew >> 2;                // which half of the subtiles
         const uint32_t acc_empty0 = mapa_shared(smem_u32(acc_empty), 0);
         uint8_t* slab0 = sEpi + ew * 2 * C::EPI_SLAB;
+        uint8_t* bias_w = smem + C::OFF_BIAS + ew * C::BIAS_WARP;
+        // Under a programmatic launch the scales and the bias may still be being written
+        // by the preceding grid: these warps read them only after it has completed.
+        griddep_wait();
         float alpha = 0.0f;
         float qg = 0.0f, qt = 0.0f;      // re-quantization: g of the next layer and 6g
+        if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
+        if constexpr (QOUT) {
+            qg = __ldg(args.q_global);
+            qt = __fmul_rn(6.0f, qg);
+        }
+        // NVFP4: this warp's bias columns of a tile, into its smem buffer (lane L: 4
+        // columns of subtile L/8); done ahead of the accumulator wait so that the load
+        // latency is not on the epilogue's path
+        auto fetch_bias = [&](int tile_, int acc_it_) {
+            if constexpr (NVF4) {
+                if (args.bias == nullptr) return;
+                const int ord = 2 * (lane >> 3) + h;
+                const int j = (acc_it_ & 1) == 0 ? (ord + 5) & 7 : ord;
+                const int n = (tile_ / num_m) * 256 + j * 32 + (lane & 7) * 4;
+                uint2 v = make_uint2(0u, 0u);
+                if (n < N) v = __ldg(reinterpret_cast<const uint2*>(args.bias + n));
+                *reinterpret_cast<uint2*>(bias_w + (lane >> 3) * 64 + (lane & 7) * 8) = v;
+            }
+        };
         const int64_t q_kb4 = N / 64;
         int acc_it = 0;
         int buf = 0;
         int committed = 0;               // bulk-store groups this warp committed
         int last_group[2] = {-1, -1};    // group that last read each slab
         const uint64_t out_policy = l2_policy_evict_first();
+        // fp8r: this lane's row scale of the next tile, also fetched ahead
+        auto fetch_sa = [&](int tile_) -> float {
+            if constexpr (NVF4) {
+                return 0.0f;
+            } else {
+                const int mrow = (tile_ % num_m) * 256 + static_cast<int>(rank) * 128 + q * 32 + lane;
+                return mrow < M ? __ldg(args.a_scale + mrow) : 0.0f;
+            }
+        };
+        float sa_next = 0.0f;
+        if (pair < num_tiles) {
+            fetch_bias(pair, 0);
+            sa_next = fetch_sa(pair);
+        }
         for (int tile = pair; tile < num_tiles; tile += npairs) {
             const int mt = tile % num_m, nt = tile / num_m;
+            __syncwarp();
             const bool ok = mbar_wait(acc_full, static_cast<uint32_t>(acc_it & 1), abort_flag,
                                       args.wait_ns, args.status, 14);
             if (!__all_sync(0xffffffffu, ok)) break;   // also reconverges the warp
             tc_fence_after();
-            // read here, after the producer's griddep_wait (through the accumulator
-            // barrier), so a preceding grid may still be writing the scales at launch
-            if constexpr (NVF4) alpha = __fmul_rn(__ldg(args.a_scale), __ldg(args.w_scale));
-            if constexpr (QOUT) {
-                qg = __ldg(args.q_global);
-                qt = __fmul_rn(6.0f, qg);
-            }
             const int sacc = acc_it & 1;
             const int wrow = mt * 256 + static_cast<int>(rank) * 128 + q * 32;   // warp's first row
             const int m = wrow + lane;
-            float sa = 0.0f;
-            if constexpr (!NVF4) sa = (m < M) ? __ldg(args.a_scale + m) : 0.0f;
+            const float sa = sa_next;
             const uint32_t tq = tbase + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(sacc * C::ACC_STRIDE);
             // Subtiles of 32 columns.  The 3 shared with the other accumulator (columns
@@ -774,7 +837,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                             for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], sa), sw[i]);
                         }
                         if (args.bias != nullptr) {
-                            const uint4 bb = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
+                            uint4 bb;
+                            if constexpr (NVF4)
+                                bb = *reinterpret_cast<const uint4*>(bias_w + idx * 64 + g * 16);
+                            else
+                                bb = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
                             const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
                             for (int i = 0; i < 4; ++i) {
@@ -832,9 +899,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 }
                 buf ^= 1;
             }
+            __syncwarp();                    // every lane has read this tile's bias
+            if (tile + npairs < num_tiles) {
+                fetch_bias(tile + npairs, acc_it + 1);
+                sa_next = fetch_sa(tile + npairs);
+            }
             ++acc_it;
         }
-        if (lane == 0) bulk_wait_group_all();
+        // the stores must have read their smem slabs before the CTA exits
+        if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
     }
 
@@ -843,7 +916,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     if (warp == 1 && lane == 0 && rank == 0) {
         tc_commit_pair(fin, 0x1);    // completes once every MMA of the pair is done
         drain_wait(fin, 0, args.wait_ns, args.status);
-        if constexpr (NVF4) drain_wait(cp_fin, 0, args.wait_ns, args.status);
+        if constexpr (NVF4)
+            if (!args.sf_inline) drain_wait(cp_fin, 0, args.wait_ns, args.status);
     }
     tc_fence_before();
     cluster_sync();
@@ -1049,6 +1123,23 @@ int kernel_choice()
     return c;
 }
 
+// NVFP4 pair kernel: who issues the scale-factor copies (1 = the MMA thread, in order
+// with the MMAs; 0 = the copy warps).  Initialised from BSP_SF_INLINE.
+std::atomic<int> g_sf_inline{-1};
+
+int sf_inline_choice()
+{
+    int c = g_sf_inline.load();
+    if (c < 0) {
+        const char* e = std::getenv("BSP_SF_INLINE");
+        c = (e && std::strcmp(e, "1") == 0) ? 1 : 0;
+        int expected = -1;
+        g_sf_inline.compare_exchange_strong(expected, c);
+        c = g_sf_inline.load();
+    }
+    return c;
+}
+
 template <bool NVF4, int BN, int STAGES, int NACC>
 int launch(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, int sms,
            cudaStream_t s, bool pdl)
@@ -1152,6 +1243,7 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     args.q_codes = q ? q->codes : nullptr;
     args.q_sf = q ? q->sf : nullptr;
     args.w_early = w_early ? 1 : 0;
+    args.sf_inline = sf_inline_choice();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (q) return launch_pair<true, true>(a, w, args, dev, sms, s, pdl);   // pair kernel only
     const int choice = kernel_choice();
