@@ -83,6 +83,16 @@ def test_nvfp4_linear_small(M, N, K, seed):
     check_nvfp4(a, w, bias)
 
 
+def test_nvfp4_bias_tiles_beyond_one_wave():
+    """80 output tiles of 256 x 256 for the 74 CTA pairs of a B200: the first pairs take
+    a second tile, which here is in the ragged last column of tiles (N = 2000), so the
+    epilogue's bias columns fetched ahead for a later tile are checked, guard included."""
+    a = synth.bf16_normal((2560, 256), 1.0, 71, 0.01, 20.0)
+    w = synth.bf16_normal((2000, 256), 0.02, 171)
+    bias = synth.bf16_normal((2000,), 0.1, 271)
+    print("nvfp4 80 tiles", check_nvfp4(a, w, bias))
+
+
 def test_nvfp4_tiny_workload():
     wl = synth.WORKLOADS["nvfp4_tiny"]
     stats = check_nvfp4(wl.A(), wl.W())
@@ -232,6 +242,15 @@ def test_fp8r_linear_small(M, N, K, seed):
     w = synth.bf16_normal((N, K), 0.02, seed + 100)
     bias = synth.bf16_normal((N,), 0.1, seed + 200) if seed % 2 == 0 else None
     check_fp8r(a, w, bias)
+
+
+def test_fp8r_bias_tiles_beyond_one_wave():
+    """As the NVFP4 case: 80 tiles for 74 pairs, the later tiles in the ragged last
+    column of tiles, with bias; the row scales of a pair's next tile are fetched ahead."""
+    a = synth.bf16_normal((2560, 256), 1.0, 72, 0.01, 20.0)
+    w = synth.bf16_normal((2000, 256), 0.02, 172)
+    bias = synth.bf16_normal((2000,), 0.1, 272)
+    print("fp8r 80 tiles", check_fp8r(a, w, bias))
 
 
 @pytest.mark.parametrize("M", synth.FP8R_M_SWEEP)
