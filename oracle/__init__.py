@@ -61,6 +61,7 @@ def lib():
         L.oracle_nvfp4_quantize.argtypes = [_u16p, _i64, _i64, ctypes.c_float, _u8p, _u8p,
                                             ctypes.c_int]
         L.oracle_nvfp4_dequant.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_double, _f64p]
+        L.oracle_nvfp4_dequant_bf16.argtypes = [_u8p, _u8p, _i64, _i64, ctypes.c_float, _u16p]
         L.oracle_fp8r_quantize.argtypes = [_u16p, _i64, _i64, _u8p, _f32p, ctypes.c_int]
         L.oracle_gemm_f64.argtypes = [_f64p, _f64p, _f64p, ctypes.c_double, _i64p, _i64,
                                       _i64, _i64, _f64p, ctypes.c_int]
@@ -170,9 +171,27 @@ def nvfp4_dequant(codes: np.ndarray, sf_lin: np.ndarray, g: float = 1.0) -> np.n
     sf_lin = np.ascontiguousarray(sf_lin, dtype=np.uint8)
     R, K2 = codes.shape
     K = 2 * K2
+    if K % 16 != 0 or sf_lin.shape != (R, K // 16):
+        raise ValueError(f"scales must be [R, K/16] = {(R, K // 16)}, got {sf_lin.shape}")
     out = np.empty((R, K), dtype=np.float64)
     lib().oracle_nvfp4_dequant(_ptr(codes, _u8p), _ptr(sf_lin, _u8p), R, K,
                                float(g), _ptr(out, _f64p))
+    return out
+
+
+def nvfp4_dequant_bf16(codes: np.ndarray, sf_lin: np.ndarray, g: float) -> np.ndarray:
+    """Decode to bf16 bit patterns (uint16 [R, K]): bf16_rne(fl32(e2m1 * e4m3) * g), the
+    weight decode of the dequantise-only fallback (closing paragraph of the "Kernels"
+    section of "BFL (fp8r / nvfp4)")."""
+    codes = np.ascontiguousarray(codes, dtype=np.uint8)
+    sf_lin = np.ascontiguousarray(sf_lin, dtype=np.uint8)
+    R, K2 = codes.shape
+    K = 2 * K2
+    if K % 16 != 0 or sf_lin.shape != (R, K // 16):
+        raise ValueError(f"scales must be [R, K/16] = {(R, K // 16)}, got {sf_lin.shape}")
+    out = np.empty((R, K), dtype=np.uint16)
+    lib().oracle_nvfp4_dequant_bf16(_ptr(codes, _u8p), _ptr(sf_lin, _u8p), R, K,
+                                    ctypes.c_float(np.float32(g)), _ptr(out, _u16p))
     return out
 
 

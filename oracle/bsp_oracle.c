@@ -272,6 +272,39 @@ void oracle_nvfp4_dequant(const uint8_t* codes, const uint8_t* sf_lin, int64_t R
         }
 }
 
+/* Dequantise to bf16, the weight decode of the dequantise-only fallback that the
+ * closing paragraph of the "Kernels" section describes (weights back to bf16, then a
+ * bf16 GEMM on activations that are not quantized).  Reading taken here: the decode
+ * is done in binary32 and rounded once to bf16, nearest-even:
+ *     p = e2m1(code) * e4m3(sb)      (exact in binary32: at most 6 significant bits)
+ *     y = p * g                      (one binary32 rounding)
+ *     out = bf16_rne(y)
+ * sf_lin is [R][K/16]; out is [R][K] bf16 bit patterns. */
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7F800000u) == 0x7F800000u && (u & 0x007FFFFFu) != 0)
+        return (uint16_t)((u >> 16) | 0x0040u);          /* NaN stays NaN (quiet) */
+    /* round to nearest, ties to even, on the 16 bits dropped */
+    uint32_t lsb = (u >> 16) & 1u;
+    uint32_t rounded = u + 0x7FFFu + lsb;
+    return (uint16_t)(rounded >> 16);
+}
+
+void oracle_nvfp4_dequant_bf16(const uint8_t* codes, const uint8_t* sf_lin, int64_t R,
+                               int64_t K, float g, uint16_t* out)
+{
+    for (int64_t r = 0; r < R; ++r)
+        for (int64_t k = 0; k < K; ++k) {
+            uint8_t byte = codes[r * (K / 2) + k / 2];
+            uint8_t c = (k % 2 == 0) ? (byte & 0xF) : (byte >> 4);
+            float p = oracle_e2m1_decode(c) * oracle_e4m3_decode(sf_lin[r * (K / 16) + k / 16]);
+            float y = p * g;
+            out[r * K + k] = f32_to_bf16_rne(y);
+        }
+}
+
 /* ------------------------------------------------------------------------- */
 /* fp8r row quantizer: q [R][K] E4M3, s [R] fp32.                             */
 /* ------------------------------------------------------------------------- */
