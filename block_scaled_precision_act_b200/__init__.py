@@ -23,7 +23,7 @@ __all__ = [
     "nvfp4_quantize_act", "nvfp4_gemm", "nvfp4_gemm_quant", "fp8r_quantize_rows", "fp8r_gemm",
     "nvfp4_linear", "nvfp4_linear_dynamic", "nvfp4_linear_workspace_bytes", "nvfp4_linear_noalloc",
     "nvfp4_linear_noalloc_max_bytes", "fp8r_linear", "fp8r_linear_workspace_bytes",
-    "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes",
+    "nvfp4_global_scale", "nvfp4_sf_convert", "nvfp4_sf_bytes", "nvfp4_dequantize",
     "bsp_last_device_status", "bsp_set_wait_limit_ms", "bsp_status_string", "bsp_version",
     "bsp_testing_gemm_stall", "bsp_testing_set_gemm_kernel", "bsp_testing_set_quant_kernel",
     "bsp_testing_cvt_range",
@@ -61,6 +61,7 @@ _SIGS = {
                   _c_int),
     "nvfp4_global_scale": ([_c_vp, _c_i64, _c_vp, _c_vp], _c_int),
     "nvfp4_sf_convert": ([_c_vp, _c_vp, _c_i64, _c_i64, _c_int, _c_int, _c_vp], _c_int),
+    "nvfp4_dequantize": ([_c_vp, _c_vp, _c_int, _c_vp, _c_i64, _c_i64, _c_vp, _c_vp], _c_int),
     "nvfp4_sf_bytes": ([_c_i64, _c_i64, _c_int], _c_i64),
     "bsp_last_device_status": ([_c_vp], _c_int),
     "bsp_set_wait_limit_ms": ([_c_i64], _c_i64),
@@ -349,6 +350,20 @@ def nvfp4_sf_convert(src, rows: int, K: int, from_layout: int, to_layout: int, d
            lib().nvfp4_sf_convert(_ptr(src), _ptr(dst), rows, K, from_layout, to_layout,
                                   _stream(stream)))
     return dst
+
+
+def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, global_scale: torch.Tensor,
+                     layout: int = SF_MMA, out=None, stream=None) -> torch.Tensor:
+    """NVFP4 codes [rows, K/2] + block scales + fp32 global scale -> bf16 [rows, K]
+    (the dequantise-only fallback's weight decode; see nvfp4_dequantize in bsp.h)."""
+    _dtype(codes, torch.uint8, "codes")
+    rows, K = codes.shape[0], 2 * codes.shape[1]
+    if out is None:
+        out = torch.empty((rows, K), dtype=torch.bfloat16, device=codes.device)
+    _check("nvfp4_dequantize",
+           lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), layout, _ptr(global_scale), rows, K,
+                                  _ptr(out), _stream(stream)))
+    return out
 
 
 def bsp_last_device_status(stream=None) -> int:

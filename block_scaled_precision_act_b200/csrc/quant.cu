@@ -415,6 +415,56 @@ __global__ void sf_to_linear_kernel(const uint8_t* __restrict__ src, uint8_t* __
     }
 }
 
+// NVFP4 -> bf16 decode (the dequantise-only fallback's weight decode): one thread per
+// 16-element block.  Per element, in binary32 with round to nearest even:
+// p = e2m1(code) * e4m3(sb) (exact), y = p * g, then one rounding to bf16.
+__device__ __forceinline__ void e2m1x2_to_f32(uint32_t byte, float& lo, float& hi)
+{
+    uint32_t h2;
+    asm("{\n\t.reg .b8 c;\n\tcvt.u8.u32 c, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, c;\n\t}"
+        : "=r"(h2)
+        : "r"(byte));
+    // element 2j sits in the low nibble and comes out in the low half
+    lo = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
+    hi = __half2float(__ushort_as_half(static_cast<unsigned short>(h2 >> 16)));
+}
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(256)
+    nvfp4_dequant_kernel(const uint2* __restrict__ codes, const uint8_t* __restrict__ scales,
+                         const float* __restrict__ gptr, uint4* __restrict__ out, int64_t nblk,
+                         int64_t nb_row)
+{
+    griddep_launch_dependents();
+    const float g = __ldg(gptr);
+    const int64_t kb4 = (nb_row + 3) >> 2;
+    for (int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; blk < nblk;
+         blk += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint2 c = __ldg(codes + blk);
+        int64_t off;
+        if (LAYOUT == BSP_SF_LINEAR) {
+            off = blk;
+        } else {
+            const int64_t row = blk / nb_row;
+            off = sf_mma_offset(row, blk - row * nb_row, kb4);
+        }
+        const float sd = e4m3_to_f32(__ldg(scales + off));
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const uint32_t byte = ((j < 4 ? c.x : c.y) >> (8 * (j & 3))) & 0xFFu;
+            float lo, hi;
+            e2m1x2_to_f32(byte, lo, hi);
+            lo = __fmul_rn(__fmul_rn(lo, sd), g);
+            hi = __fmul_rn(__fmul_rn(hi, sd), g);
+            __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
+            w[j] = *reinterpret_cast<uint32_t*>(&b);
+        }
+        out[2 * blk] = make_uint4(w[0], w[1], w[2], w[3]);
+        out[2 * blk + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+}
+
 // NVFP4 quantizer kernel choice: 0 = by size, 1 = grid-stride, 2 = staged (test hook)
 std::atomic<int> g_quant_choice{0};
 
@@ -601,6 +651,36 @@ int nvfp4_global_scale(const void* x_bf16, int64_t n, float* global_scale_out,
         if (st != BSP_OK) return st;
     }
     global_scale_finalize_kernel<<<1, 1, 0, s>>>(global_scale_out);
+    return launch_status();
+}
+
+int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int layout,
+                     const float* global_scale, int64_t rows, int64_t K, void* out_bf16,
+                     bsp_stream_t stream)
+{
+    using namespace bsp;
+    if (rows < 0 || K <= 0 || (layout != BSP_SF_LINEAR && layout != BSP_SF_MMA))
+        return BSP_ERR_INVALID_ARG;
+    if (rows == 0) return BSP_OK;
+    if (!codes || !scales || !global_scale || !out_bf16) return BSP_ERR_INVALID_ARG;
+    if (K % 16 != 0 || (layout == BSP_SF_MMA && K % 64 != 0)) return BSP_ERR_UNSUPPORTED_SHAPE;
+    if (!aligned16(codes) || !aligned16(out_bf16) ||
+        (reinterpret_cast<uintptr_t>(global_scale) & 3u))
+        return BSP_ERR_MISALIGNED;
+    int dev = 0, sms = 0;
+    int st = check_device(&dev, &sms);
+    if (st != BSP_OK) return st;
+    const int64_t nblk = rows * (K / 16);
+    const int grid = grid_for(nblk, 256, sms, 8);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const auto* cv = reinterpret_cast<const uint2*>(codes);
+    auto* ov = static_cast<uint4*>(out_bf16);
+    if (layout == BSP_SF_LINEAR)
+        nvfp4_dequant_kernel<BSP_SF_LINEAR><<<grid, 256, 0, s>>>(cv, scales, global_scale, ov,
+                                                                  nblk, K / 16);
+    else
+        nvfp4_dequant_kernel<BSP_SF_MMA><<<grid, 256, 0, s>>>(cv, scales, global_scale, ov,
+                                                               nblk, K / 16);
     return launch_status();
 }
 

@@ -262,6 +262,28 @@ int nvfp4_global_scale(const void* x_bf16, int64_t n, float* global_scale_out,
                        bsp_stream_t stream);
 
 /*
+ * nvfp4_dequantize -- decode NVFP4 to bf16: the weight decode of the dequantise-only
+ * fallback ("BFL (fp8r / nvfp4)", closing paragraph of the "Kernels" section: weights are
+ * dequantized back to bf16 and the GEMM runs in bf16 on activations that are not
+ * quantized, so results differ slightly from the fused path).  Per element, in binary32
+ * with round to nearest even and no flush to zero:
+ *     out = bf16_rne( (e2m1(code) * e4m3(scale)) * g )
+ * (the first product is exact).  Not on the fused hot path; provided for comparison and
+ * for callers that need bf16 weights.
+ *   codes         [rows][K/2] packed E2M1 (element 2j in the low nibble)
+ *   scales        E4M3 block scales in `layout` (BSP_SF_LINEAR [rows][K/16] or BSP_SF_MMA)
+ *   global_scale  device fp32, 1 element (weight_scale_2 or input_scale)
+ *   out_bf16      [rows][K] bf16, caller-owned
+ * Constraints: K % 16 == 0 (K % 64 == 0 for BSP_SF_MMA); codes and out 16-byte aligned,
+ * global_scale 4-byte aligned; scale bytes finite (a NaN scale gives NaN elements).
+ * Errors: BSP_ERR_INVALID_ARG, BSP_ERR_UNSUPPORTED_SHAPE, BSP_ERR_MISALIGNED,
+ * BSP_ERR_UNSUPPORTED_DEVICE, BSP_ERR_CUDA.  Asynchronous on `stream`; no allocation.
+ */
+int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int layout,
+                     const float* global_scale, int64_t rows, int64_t K, void* out_bf16,
+                     bsp_stream_t stream);
+
+/*
  * nvfp4_sf_convert -- re-lay block scales between BSP_SF_LINEAR and BSP_SF_MMA
  * (rows x K/16 bytes; padding of an MMA-layout destination is written as 0).
  * Constraints: K % 64 == 0.  src and dst must not overlap.

@@ -82,6 +82,19 @@ def test_quantize_validation_on_host():
     assert g(None, 16, P, None) == INVALID
 
 
+def test_dequantize_validation_on_host():
+    d = bsp.lib().nvfp4_dequantize
+    assert d(None, P, 1, P, 8, 64, P, None) == INVALID
+    assert d(P, P, 7, P, 8, 64, P, None) == INVALID            # unknown layout
+    assert d(P, P, 1, P, -1, 64, P, None) == INVALID
+    assert d(P, P, 0, P, 8, 24, P, None) == SHAPE              # K % 16
+    assert d(P, P, 1, P, 8, 80, P, None) == SHAPE              # MMA layout needs K % 64
+    assert d(P + 8, P, 1, P, 8, 64, P, None) == MISALIGNED
+    assert d(P, P, 1, P + 2, 8, 64, P, None) == MISALIGNED     # fp32 scalar alignment
+    assert d(P, P, 1, P, 8, 64, P + 4, None) == MISALIGNED
+    assert d(P, P, 1, P, 0, 64, P, None) == 0                  # nothing to do
+
+
 def test_gemm_validation_on_host():
     L = bsp.lib()
     n = L.nvfp4_gemm
