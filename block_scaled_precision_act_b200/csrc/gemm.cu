@@ -818,6 +818,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     tmem_ld_wait();
                 }
                 uint32_t packed[16];
+                if (NVF4 && n0 + 32 <= N) {
+                    // whole subtile inside N: the four bias reads go out before the math
+                    uint4 bb[4];
+                    const bool has_bias = args.bias != nullptr;
+                    if (has_bias) {
+#pragma unroll
+                        for (int g = 0; g < 4; ++g)
+                            bb[g] = *reinterpret_cast<const uint4*>(bias_w + idx * 64 + g * 16);
+                    }
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            v[i] = __fmul_rn(__uint_as_float(r[g * 8 + i]), alpha);
+                        if (has_bias) {
+                            const uint32_t bw[4] = {bb[g].x, bb[g].y, bb[g].z, bb[g].w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                v[2 * i] = __fadd_rn(v[2 * i], bf16lo_to_f32(bw[i]));
+                                v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16hi_to_f32(bw[i]));
+                            }
+                        }
+#pragma unroll
+                        for (int i = 0; i < 4; ++i)
+                            packed[g * 4 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                    }
+                } else
 #pragma unroll
                 for (int g = 0; g < 4; ++g) {
                     const int n = n0 + g * 8;
