@@ -148,6 +148,25 @@ class ClockSampler:
                 "reasons": names, "samples": len(self.samples)}
 
 
+# ---------------------------------------------------------------------- replicas (N > 1)
+def max_over_ranks(value: float, device) -> float:
+    """MAX of a per-rank timing over all ranks of the default process group (the value
+    itself when there is no group or it has one rank).  Every rank must call it."""
+    import torch
+    import torch.distributed as dist
+    if not dist.is_available() or not dist.is_initialized() or dist.get_world_size() == 1:
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def replica_tflops(flops_per_step: float, ms_per_step: float, world: int) -> float:
+    """Whole-job throughput of `world` independent replicas, each doing `flops_per_step`
+    per step, timed by the slowest rank's `ms_per_step`."""
+    return world * flops_per_step / (ms_per_step * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------------- CPU oracle
 def cpu_oracle_sample(wl, rows: int, A=None, W=None):
     """Quantize `rows` rows of A and run the fp64 GEMM against the full weight with the
@@ -381,10 +400,7 @@ def run_bsp(args):
     total_ms = sum(s_ms)
     part_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in kev)
                for j in range(len(parts))]
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dev)
     if bsp.bsp_last_device_status() != 0:
         raise SystemExit("device status not OK after the timed steps")
     if not torch.isfinite(y_out.float()).all():
@@ -403,10 +419,7 @@ def run_bsp(args):
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
 
     ms_per_step = total_ms / args.steps
     kernels = {}
@@ -432,7 +445,7 @@ def run_bsp(args):
                      "GEMM as programmatic dependent)")
     line = {
         "metric": METRIC,
-        "value": world * flops / (ms_per_step * 1e-3) / 1e12,
+        "value": replica_tflops(flops, ms_per_step, world),
         "unit": "TFLOP/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -449,7 +462,7 @@ def run_bsp(args):
                                     f"{pk['bf16_tflops']} TFLOP/s (nominal dense "
                                     f"{'fp4' if nvf4 else 'fp8'}:bf16 = {4 if nvf4 else 2})"},
         "kernels": kernels,
-        "e2e": {"value": world * flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        "e2e": {"value": replica_tflops(flops, e2e_ms, world), "unit": "TFLOP/s",
                 "h2d_bytes_per_step": M * K * 2, "d2h_bytes_per_step": y_out.numel() * 2},
         "gpu_launches": len(parts) * args.steps,
         "clocks": sampler.summary(),
