@@ -25,6 +25,20 @@ int gemm_after_quantizer(bool nvf4, const uint8_t* a, const uint8_t* a_sf, const
                          const void* bias_bf16, void* out_bf16, int64_t M, int64_t N, int64_t K,
                          bsp_stream_t stream);
 
+// nvfp4_quantize_act with an optional per-call global scale: when `partials` is not null,
+// g is reduced from the `npartials` per-CTA maxima of |x| there (fp32 bit patterns) and
+// published at `gout`; `global_scale` is then unused.
+int quantize_act_impl(const void* x_bf16, int64_t M, int64_t K, const float* global_scale,
+                      uint8_t* codes, uint8_t* scales, int layout, bsp_stream_t stream,
+                      const uint32_t* partials, int npartials, float* gout);
+
+// Slots of per-CTA maxima the dynamic path keeps in the linear workspace.
+constexpr int kDynamicPartials = 2048;
+
+// amax pass into `partials`, then the quantizer reducing them (MMA scale layout).
+int dynamic_quantize_front(const void* x_bf16, int64_t M, int64_t K, uint32_t* partials,
+                           float* g_out, uint8_t* codes, uint8_t* scales, bsp_stream_t stream);
+
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 inline int launch_status()

@@ -21,6 +21,12 @@ int64_t scales_offset(int64_t M, int64_t K)
 
 int64_t align_up(int64_t v) { return (v + kWorkspaceAlign - 1) / kWorkspaceAlign * kWorkspaceAlign; }
 
+// after the scales, at a 256-byte boundary: the dynamic path's per-CTA maxima
+int64_t partials_offset(int64_t M, int64_t K)
+{
+    return align_up(scales_offset(M, K) + nvfp4_sf_bytes(M, K, BSP_SF_MMA));
+}
+
 }  // namespace
 }  // namespace bsp
 
@@ -32,7 +38,7 @@ int64_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K)
     if (M > (int64_t{1} << 40) / K) return BSP_ERR_UNSUPPORTED_SHAPE;
     const int64_t sf = nvfp4_sf_bytes(M, K, BSP_SF_MMA);
     if (sf < 0) return sf;
-    return bsp::scales_offset(M, K) + sf;
+    return bsp::partials_offset(M, K) + bsp::kDynamicPartials * 4;
 }
 
 int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_codes,
@@ -69,11 +75,18 @@ int nvfp4_linear_dynamic(const void* x_bf16, float* input_scale_out, const uint8
     const int64_t need = nvfp4_linear_workspace_bytes(M, K);
     if (need < 0) return static_cast<int>(need);
     if (!workspace || workspace_bytes < need) return BSP_ERR_INVALID_ARG;
-    // g = amax(x) / (448 * 6) of this very activation, then the static-scale path with it
-    int st = nvfp4_global_scale(x_bf16, M * K, input_scale_out, stream);
+    if (!bsp::aligned16(workspace)) return BSP_ERR_MISALIGNED;
+    if (reinterpret_cast<uintptr_t>(input_scale_out) & 3u) return BSP_ERR_MISALIGNED;
+    // g = amax(x) / (448 * 6) of this very activation: per-CTA maxima into the workspace,
+    // reduced by the quantizer's CTAs, which also publish g for the GEMM
+    auto* a_codes = static_cast<uint8_t*>(workspace);
+    uint8_t* a_sf = a_codes + bsp::scales_offset(M, K);
+    auto* partials = reinterpret_cast<uint32_t*>(a_codes + bsp::partials_offset(M, K));
+    int st = bsp::dynamic_quantize_front(x_bf16, M, K, partials, input_scale_out, a_codes, a_sf,
+                                        stream);
     if (st != BSP_OK) return st;
-    return nvfp4_linear(x_bf16, input_scale_out, w_codes, w_sf, w_scale, bias_bf16, out_bf16, M,
-                        N, K, workspace, workspace_bytes, stream);
+    return bsp::gemm_after_quantizer(true, a_codes, a_sf, input_scale_out, w_codes, w_sf, w_scale,
+                                     bias_bf16, out_bf16, M, N, K, stream);
 }
 
 int64_t fp8r_linear_workspace_bytes(int64_t M, int64_t K)

@@ -131,16 +131,44 @@ __device__ __forceinline__ void store_block(uint2* codes, uint8_t* scales, int64
     }
 }
 
+// The kernel's global scale g.  Static: the fp32 at gptr.  Dynamic (partials != null):
+// the per-CTA maxima of |x| that amax_kernel left as fp32 bit patterns are reduced here by
+// every CTA, g = amax / (448 * 6) (one binary32 division, as nvfp4_global_scale), and CTA 0
+// publishes g at gout for the GEMM that follows.  Every thread of the CTA must call it.
+__device__ __forceinline__ float resolve_global_scale(const float* gptr, const uint32_t* partials,
+                                                      int npartials, float* gout)
+{
+    if (partials == nullptr) return __ldg(gptr);
+    __shared__ uint32_t red[32];
+    uint32_t m = 0;
+    for (int i = threadIdx.x; i < npartials; i += blockDim.x) m = max(m, __ldg(partials + i));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        m = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0u;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+        if (threadIdx.x == 0) red[0] = m;
+    }
+    __syncthreads();
+    const float g = __fdiv_rn(__uint_as_float(red[0]), 2688.0f);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *gout = g;
+    return g;
+}
+
 template <int LAYOUT, bool IDX32>
 __global__ void __launch_bounds__(kQuantThreads)
     nvfp4_quant_kernel(const uint4* __restrict__ x, int64_t nblk, int64_t nb_row, RowDiv rd,
                        const float* __restrict__ gptr, uint2* __restrict__ codes,
-                       uint8_t* __restrict__ scales)
+                       uint8_t* __restrict__ scales, const uint32_t* __restrict__ partials,
+                       int npartials, float* gout)
 {
     // a GEMM launched as this grid's programmatic dependent may start its prologue now;
     // it still waits for this grid to complete before reading the codes
     griddep_launch_dependents();
-    const float g = __ldg(gptr);
+    const float g = resolve_global_scale(gptr, partials, npartials, gout);
     const float t = __fmul_rn(6.0f, g);
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
@@ -194,11 +222,13 @@ __global__ void __launch_bounds__(kStageThreads, 1)
     nvfp4_quant_staged_kernel(const uint8_t* __restrict__ x, int64_t nblk, int64_t nb_row,
                               RowDiv rd, const float* __restrict__ gptr, uint2* __restrict__ codes,
                               uint8_t* __restrict__ scales, int64_t blocks_per_cta, int* status,
-                              uint64_t wait_ns)
+                              uint64_t wait_ns, const uint32_t* __restrict__ partials,
+                              int npartials, float* gout)
 {
     // a GEMM launched as this grid's programmatic dependent may start its prologue now;
     // it still waits for this grid to complete before reading the codes
     griddep_launch_dependents();
+    const float g_cta = resolve_global_scale(gptr, partials, npartials, gout);
     extern __shared__ uint8_t smem_raw[];
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) &
                                                ~uintptr_t(127));
@@ -240,7 +270,7 @@ __global__ void __launch_bounds__(kStageThreads, 1)
                            wait_ns, status);
         }
     } else {
-        const float g = __ldg(gptr);
+        const float g = g_cta;
         const float t = __fmul_rn(6.0f, g);
         const int64_t kb4 = (nb_row + 3) >> 2;
         const int cw = warp - 1;
@@ -360,27 +390,52 @@ __global__ void __launch_bounds__(kRowThreads)
 }
 
 // ---------------------------------------------------------------- global scale
+// amax(|x|) over bf16 values, as the bit pattern of a non-negative fp32 (atomic max on
+// *out, which the caller clears first).  Each thread keeps four 16-byte loads in flight
+// and takes the max on the sign-cleared bf16 bit patterns (max.bf16x2, starting from 0 so
+// a NaN loses as with fmaxf); the largest |x| is exact in bf16, so the result is the
+// binary32 max of |x|.
+template <bool PARTIAL>
 __global__ void __launch_bounds__(256)
     amax_kernel(const uint4* __restrict__ x, int64_t n8, unsigned int* __restrict__ out)
 {
-    __shared__ float red[8];
-    float m = 0.0f;
-    for (int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x; i < n8;
-         i += static_cast<int64_t>(gridDim.x) * 256) {
-        float f[8];
-        unpack8(ld_stream(x + i), f);
+    __shared__ uint32_t red[8];
+    uint32_t m2 = 0;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * 256;
+    int64_t i = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+    for (; i + 3 * stride < n8; i += 4 * stride) {
+        uint4 v[4];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m = fmaxf(m, fabsf(f[e]));
+        for (int u = 0; u < 4; ++u) v[u] = ld_stream(x + i + u * stride);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            m2 = max_bf16x2(m2, v[u].x & 0x7FFF7FFFu);
+            m2 = max_bf16x2(m2, v[u].y & 0x7FFF7FFFu);
+            m2 = max_bf16x2(m2, v[u].z & 0x7FFF7FFFu);
+            m2 = max_bf16x2(m2, v[u].w & 0x7FFF7FFFu);
+        }
     }
+    for (; i < n8; i += stride) {
+        const uint4 v = ld_stream(x + i);
+        m2 = max_bf16x2(m2, v.x & 0x7FFF7FFFu);
+        m2 = max_bf16x2(m2, v.y & 0x7FFF7FFFu);
+        m2 = max_bf16x2(m2, v.z & 0x7FFF7FFFu);
+        m2 = max_bf16x2(m2, v.w & 0x7FFF7FFFu);
+    }
+    m2 = max_bf16x2(m2, __byte_perm(m2, 0, 0x1032));
+    uint32_t m = m2 << 16;                       // fp32 bits of the larger |x|
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
     if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
     __syncthreads();
     if (threadIdx.x == 0) {
-        float b = red[0];
-        for (int w = 1; w < 8; ++w) b = fmaxf(b, red[w]);
+        uint32_t b = red[0];
+        for (int w = 1; w < 8; ++w) b = max(b, red[w]);
         // non-negative floats order like their bit patterns
-        atomicMax(out, __float_as_uint(b));
+        if (PARTIAL)
+            out[blockIdx.x] = b;           // one slot per CTA, reduced by the quantizer
+        else
+            atomicMax(out, b);
     }
 }
 
@@ -499,7 +554,18 @@ extern "C" {
 int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* global_scale,
                        uint8_t* codes, uint8_t* scales, int layout, bsp_stream_t stream)
 {
-    using namespace bsp;
+    return bsp::quantize_act_impl(x_bf16, M, K, global_scale, codes, scales, layout, stream,
+                                  nullptr, 0, nullptr);
+}
+
+}  // extern "C"
+
+namespace bsp {
+
+int quantize_act_impl(const void* x_bf16, int64_t M, int64_t K, const float* global_scale,
+                      uint8_t* codes, uint8_t* scales, int layout, bsp_stream_t stream,
+                      const uint32_t* partials, int npartials, float* gout)
+{
     if (M < 0 || K <= 0 || (layout != BSP_SF_LINEAR && layout != BSP_SF_MMA))
         return BSP_ERR_INVALID_ARG;
     if (M == 0) return BSP_OK;
@@ -530,13 +596,13 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
             nblk + static_cast<int64_t>(grid) * kQuantThreads * 2 < (int64_t{1} << 31);
         if (layout == BSP_SF_LINEAR)
             nvfp4_quant_kernel<BSP_SF_LINEAR, false><<<grid, kQuantThreads, 0, s>>>(
-                xv, nblk, K / 16, rd, global_scale, cv, scales);
+                xv, nblk, K / 16, rd, global_scale, cv, scales, partials, npartials, gout);
         else if (idx32)
             nvfp4_quant_kernel<BSP_SF_MMA, true><<<grid, kQuantThreads, 0, s>>>(
-                xv, nblk, K / 16, rd, global_scale, cv, scales);
+                xv, nblk, K / 16, rd, global_scale, cv, scales, partials, npartials, gout);
         else
             nvfp4_quant_kernel<BSP_SF_MMA, false><<<grid, kQuantThreads, 0, s>>>(
-                xv, nblk, K / 16, rd, global_scale, cv, scales);
+                xv, nblk, K / 16, rd, global_scale, cv, scales, partials, npartials, gout);
         return launch_status();
     }
     // one persistent CTA per SM, each a contiguous range of whole 64-block warp spans
@@ -563,15 +629,44 @@ int nvfp4_quantize_act(const void* x_bf16, int64_t M, int64_t K, const float* gl
     const uint64_t wns = wait_limit_ns();
     if (layout == BSP_SF_LINEAR)
         nvfp4_quant_staged_kernel<BSP_SF_LINEAR, false><<<grid, kStageThreads, kStageSmem, s>>>(
-            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
+            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns, partials,
+            npartials, gout);
     else if (idx32)
         nvfp4_quant_staged_kernel<BSP_SF_MMA, true><<<grid, kStageThreads, kStageSmem, s>>>(
-            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
+            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns, partials,
+            npartials, gout);
     else
         nvfp4_quant_staged_kernel<BSP_SF_MMA, false><<<grid, kStageThreads, kStageSmem, s>>>(
-            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns);
+            xb, nblk, K / 16, rd, global_scale, cv, scales, bpc, status, wns, partials,
+            npartials, gout);
     return launch_status();
 }
+
+// The nvfp4 front half of a linear with a per-call activation scale: per-CTA maxima of |x|
+// into `partials` (at most kDynamicPartials slots), then the quantizer, whose CTAs reduce
+// them to g = amax / (448 * 6) and publish g at `g_out`.  Two launches, no clear.
+int dynamic_quantize_front(const void* x_bf16, int64_t M, int64_t K, uint32_t* partials,
+                           float* g_out, uint8_t* codes, uint8_t* scales, bsp_stream_t stream)
+{
+    if (M <= 0 || K <= 0 || K % 64 != 0 || !x_bf16 || !partials || !g_out) return BSP_ERR_INVALID_ARG;
+    if (!aligned16(x_bf16)) return BSP_ERR_MISALIGNED;
+    int dev = 0, sms = 0;
+    int st = check_device(&dev, &sms);
+    if (st != BSP_OK) return st;
+    const int64_t n8 = M * K / 8;
+    int grid = grid_for(n8, 256 * 4, sms, 8);
+    if (grid > kDynamicPartials) grid = kDynamicPartials;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    amax_kernel<true><<<grid, 256, 0, s>>>(static_cast<const uint4*>(x_bf16), n8, partials);
+    st = launch_status();
+    if (st != BSP_OK) return st;
+    return quantize_act_impl(x_bf16, M, K, g_out, codes, scales, BSP_SF_MMA, stream, partials, grid,
+                             g_out);
+}
+
+}  // namespace bsp
+
+extern "C" {
 
 int bsp_testing_cvt_range(int kind, uint32_t first, int64_t n, uint8_t* out, bsp_stream_t stream)
 {
@@ -644,8 +739,8 @@ int nvfp4_global_scale(const void* x_bf16, int64_t n, float* global_scale_out,
         return BSP_ERR_CUDA;
     }
     if (n > 0) {
-        const int grid = grid_for(n / 8, 256 * 4, sms, 4);
-        amax_kernel<<<grid, 256, 0, s>>>(static_cast<const uint4*>(x_bf16), n / 8,
+        const int grid = grid_for(n / 8, 256 * 4, sms, 8);
+        amax_kernel<false><<<grid, 256, 0, s>>>(static_cast<const uint4*>(x_bf16), n / 8,
                                          reinterpret_cast<unsigned int*>(global_scale_out));
         st = launch_status();
         if (st != BSP_OK) return st;

@@ -148,9 +148,11 @@ int nvfp4_gemm_quant(const uint8_t* a_codes, const uint8_t* a_sf, const float* a
  *   bias_bf16     [N] bf16 or NULL.   out_bf16  [M][N] bf16.
  *   workspace     caller-owned device buffer of at least
  *                 nvfp4_linear_workspace_bytes(M, K) bytes, 16-byte aligned.  It receives
- *                 the quantized activations (codes, then scales at a 256-byte boundary),
- *                 is fully overwritten by every call, and must not be in use by another
- *                 call that can run at the same time (another stream).
+ *                 the quantized activations (codes, then scales at a 256-byte boundary;
+ *                 after them, at the next 256-byte boundary, 8 KB that
+ *                 nvfp4_linear_dynamic uses for per-CTA maxima), is overwritten by every
+ *                 call, and must not be in use by another call that can run at the same
+ *                 time (another stream).
  * Constraints: K % 64 == 0, K >= 64, N % 8 == 0 (those of the two calls).
  * Errors: BSP_ERR_INVALID_ARG when workspace is NULL or workspace_bytes too small;
  * otherwise as nvfp4_quantize_act and nvfp4_gemm.
@@ -164,19 +166,22 @@ int nvfp4_linear(const void* x_bf16, const float* input_scale, const uint8_t* w_
  * nvfp4_linear_dynamic -- nvfp4_linear with the activation global scale computed from
  * this call's activations instead of a calibrated constant ("BFL (fp8r / nvfp4)",
  * nvfp4 bullet: `input_scale` is an fp32 activation scale; here g = amax(x) / (448*6),
- * the global-scale convention used for the weights): nvfp4_global_scale(x) into
- * *input_scale_out, then nvfp4_linear with it.  input_scale_out is a device fp32 the
- * caller owns; it holds g when the call's work completes.  Other arguments, workspace
- * rules and errors as nvfp4_linear.  Costs one more read of x (an atomic-max pass) than
- * nvfp4_linear.
+ * the global-scale convention used for the weights, the same value nvfp4_global_scale(x)
+ * gives), then the nvfp4_linear path with it.  Two launches precede the GEMM: a pass over
+ * x leaving one maximum of |x| per CTA in the workspace, and the quantizer, whose CTAs
+ * reduce those maxima to g themselves; CTA 0 writes g to *input_scale_out, which the GEMM
+ * then reads.  input_scale_out is a device fp32 the caller owns (4-byte aligned); it holds
+ * g when the call's work completes.  Other arguments, workspace rules and errors as
+ * nvfp4_linear.  Costs one more read of x than nvfp4_linear.
  */
 int nvfp4_linear_dynamic(const void* x_bf16, float* input_scale_out, const uint8_t* w_codes,
                          const uint8_t* w_sf, const float* w_scale, const void* bias_bf16,
                          void* out_bf16, int64_t M, int64_t N, int64_t K, void* workspace,
                          int64_t workspace_bytes, bsp_stream_t stream);
 
-/* Workspace bytes nvfp4_linear needs for an [M][K] activation (codes, padding to 256
- * bytes, MMA-layout scales); negative on bad arguments. */
+/* Workspace bytes nvfp4_linear / nvfp4_linear_dynamic need for an [M][K] activation
+ * (codes, padding to 256 bytes, MMA-layout scales, padding to 256 bytes, 8 KB of per-CTA
+ * maxima); negative on bad arguments. */
 int64_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
 
 /*

@@ -117,7 +117,8 @@ def test_linear_workspace_and_validation_on_host():
     L = bsp.lib()
     for M, K in [(1, 64), (4096, 3072), (200, 320), (0, 128)]:
         codes = M * K // 2
-        expect = (codes + 255) // 256 * 256 + oracle.sf_bytes(M, K, True)
+        scales_end = (codes + 255) // 256 * 256 + oracle.sf_bytes(M, K, True)
+        expect = (scales_end + 255) // 256 * 256 + 8192      # + per-CTA maxima (dynamic)
         assert bsp.nvfp4_linear_workspace_bytes(M, K) == expect
     assert L.nvfp4_linear_workspace_bytes(128, 96) == INVALID
     assert L.nvfp4_linear_workspace_bytes(-1, 64) == INVALID
