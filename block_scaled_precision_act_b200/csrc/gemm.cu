@@ -65,9 +65,6 @@ struct GemmArgs {
     // on, so the pair producer may fetch the first stages of it before griddep_wait
     // (set only where that grid is the library's own activation quantizer)
     int w_early;
-    // pair kernel, NVFP4: the MMA thread issues each stage's scale-factor copies itself,
-    // in order ahead of the stage's MMAs, instead of the copy warps
-    int sf_inline;
 };
 
 template <bool NVF4, int BN, int STAGES, int NACC>
@@ -607,38 +604,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     }
                     int nk;
                     if constexpr (NVF4) {
-                        if (args.sf_inline) {
-                            // the stage's scale copies go into the pair's in-order tensor
-                            // queue just ahead of the MMAs that read them
-                            if (!mbar_wait(full + s, ph, abort_flag, args.wait_ns, args.status,
-                                           13)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            nk = min(4, K / 64 - 4 * kt);
-                            const uint32_t sfd = tbase + C::SF_COL0 + b * C::SF_BUF;
-                            for (int kb = 0; kb < nk; ++kb) {
-                                tmem_cp_32x128b_x4_pair(
-                                    sfd + kb * 4,
-                                    sdesc_sf_block(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512)));
-                                tmem_cp_32x128b_x4_pair(
-                                    sfd + 16 + kb * 8,
-                                    sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES + kb * 512)));
-                                tmem_cp_32x128b_x4_pair(
-                                    sfd + 16 + kb * 8 + 4,
-                                    sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES + 2048 +
-                                                            kb * 512)));
-                            }
-                        } else {
-                            if (!mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status,
-                                           15)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            nk = min(4, K / 64 - 4 * kt);
+                        if (!mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status,
+                                       15)) {
+                            ok = false;
+                            break;
                         }
+                        tc_fence_after();
+                        nk = min(4, K / 64 - 4 * kt);
                     } else {
                         nk = min(4 * C::ATOMS, (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
                     }
@@ -658,8 +630,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                             mma_f8f6f4_pair(d_tmem, adesc + koff, bdesc + koff, C::IDESC, acc);
                     }
                     tc_commit_pair(empty + s, 0x1);
-                    if constexpr (NVF4)
-                        if (!args.sf_inline) tc_commit_pair(sf_empty + b, 0x1);
+                    if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -675,7 +646,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     } else if (warp <= 4) {
         // ------------------------------------------------------------ scale copies (CTA 0)
         if constexpr (NVF4) {
-            if (lane == 0 && rank == 0 && !args.sf_inline) {
+            if (lane == 0 && rank == 0) {
                 const int which = warp - 2;          // 0: SFA, 1: SFB rows 0-127, 2: rows 128-255
                 int s = 0;
                 uint32_t ph = 0;
@@ -944,8 +915,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     if (warp == 1 && lane == 0 && rank == 0) {
         tc_commit_pair(fin, 0x1);    // completes once every MMA of the pair is done
         drain_wait(fin, 0, args.wait_ns, args.status);
-        if constexpr (NVF4)
-            if (!args.sf_inline) drain_wait(cp_fin, 0, args.wait_ns, args.status);
+        if constexpr (NVF4) drain_wait(cp_fin, 0, args.wait_ns, args.status);
     }
     tc_fence_before();
     cluster_sync();
@@ -1151,23 +1121,6 @@ int kernel_choice()
     return c;
 }
 
-// NVFP4 pair kernel: who issues the scale-factor copies (1 = the MMA thread, in order
-// with the MMAs; 0 = the copy warps).  Initialised from BSP_SF_INLINE.
-std::atomic<int> g_sf_inline{-1};
-
-int sf_inline_choice()
-{
-    int c = g_sf_inline.load();
-    if (c < 0) {
-        const char* e = std::getenv("BSP_SF_INLINE");
-        c = (e && std::strcmp(e, "1") == 0) ? 1 : 0;
-        int expected = -1;
-        g_sf_inline.compare_exchange_strong(expected, c);
-        c = g_sf_inline.load();
-    }
-    return c;
-}
-
 template <bool NVF4, int BN, int STAGES, int NACC>
 int launch(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, int sms,
            cudaStream_t s, bool pdl)
@@ -1271,7 +1224,6 @@ int gemm_entry(bool nvf4, const uint8_t* a, const uint8_t* sfa, const float* a_s
     args.q_codes = q ? q->codes : nullptr;
     args.q_sf = q ? q->sf : nullptr;
     args.w_early = w_early ? 1 : 0;
-    args.sf_inline = sf_inline_choice();
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (q) return launch_pair<true, true>(a, w, args, dev, sms, s, pdl);   // pair kernel only
     const int choice = kernel_choice();
