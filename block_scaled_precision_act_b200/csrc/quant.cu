@@ -486,16 +486,19 @@ __device__ __forceinline__ void e2m1x2_to_f32(uint32_t byte, float& lo, float& h
 
 template <int LAYOUT>
 __global__ void __launch_bounds__(256)
-    nvfp4_dequant_kernel(const uint2* __restrict__ codes, const uint8_t* __restrict__ scales,
-                         const float* __restrict__ gptr, uint4* __restrict__ out, int64_t nblk,
+    nvfp4_dequant_kernel(const uint32_t* __restrict__ codes, const uint8_t* __restrict__ scales,
+                         const float* __restrict__ gptr, uint4* __restrict__ out, int64_t nhalf,
                          int64_t nb_row)
 {
+    // one thread per half block (8 elements): 4 code bytes in, 16 bytes of bf16 out, so a
+    // warp's loads and stores are both contiguous
     griddep_launch_dependents();
     const float g = __ldg(gptr);
     const int64_t kb4 = (nb_row + 3) >> 2;
-    for (int64_t blk = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; blk < nblk;
-         blk += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const uint2 c = __ldg(codes + blk);
+    for (int64_t h = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; h < nhalf;
+         h += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const uint32_t c = __ldg(codes + h);
+        const int64_t blk = h >> 1;
         int64_t off;
         if (LAYOUT == BSP_SF_LINEAR) {
             off = blk;
@@ -504,19 +507,17 @@ __global__ void __launch_bounds__(256)
             off = sf_mma_offset(row, blk - row * nb_row, kb4);
         }
         const float sd = e4m3_to_f32(__ldg(scales + off));
-        uint32_t w[8];
+        uint32_t w[4];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const uint32_t byte = ((j < 4 ? c.x : c.y) >> (8 * (j & 3))) & 0xFFu;
+        for (int j = 0; j < 4; ++j) {
             float lo, hi;
-            e2m1x2_to_f32(byte, lo, hi);
+            e2m1x2_to_f32((c >> (8 * j)) & 0xFFu, lo, hi);
             lo = __fmul_rn(__fmul_rn(lo, sd), g);
             hi = __fmul_rn(__fmul_rn(hi, sd), g);
             __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
             w[j] = *reinterpret_cast<uint32_t*>(&b);
         }
-        out[2 * blk] = make_uint4(w[0], w[1], w[2], w[3]);
-        out[2 * blk + 1] = make_uint4(w[4], w[5], w[6], w[7]);
+        out[h] = make_uint4(w[0], w[1], w[2], w[3]);
     }
 }
 
@@ -765,17 +766,17 @@ int nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, int layout,
     int dev = 0, sms = 0;
     int st = check_device(&dev, &sms);
     if (st != BSP_OK) return st;
-    const int64_t nblk = rows * (K / 16);
-    const int grid = grid_for(nblk, 256, sms, 8);
+    const int64_t nhalf = rows * (K / 8);
+    const int grid = grid_for(nhalf, 256 * 2, sms, 8);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const auto* cv = reinterpret_cast<const uint2*>(codes);
+    const auto* cv = reinterpret_cast<const uint32_t*>(codes);
     auto* ov = static_cast<uint4*>(out_bf16);
     if (layout == BSP_SF_LINEAR)
         nvfp4_dequant_kernel<BSP_SF_LINEAR><<<grid, 256, 0, s>>>(cv, scales, global_scale, ov,
-                                                                  nblk, K / 16);
+                                                                  nhalf, K / 16);
     else
         nvfp4_dequant_kernel<BSP_SF_MMA><<<grid, 256, 0, s>>>(cv, scales, global_scale, ov,
-                                                               nblk, K / 16);
+                                                               nhalf, K / 16);
     return launch_status();
 }
 

@@ -130,3 +130,45 @@ def test_linear_dynamic_scale():
     y2, g2 = bsp.nvfp4_linear_dynamic(a * 4, wc, wsf, gw)
     torch.cuda.synchronize()
     assert g2.item() == 4 * g.item()
+
+
+@pytest.mark.parametrize("kernel", [1, 2])        # grid-stride / staged quantizer
+@pytest.mark.parametrize("M,N,K", [(300, 512, 1024), (1, 8, 64), (4096, 256, 3072)])
+def test_linear_dynamic_scale_both_quantizer_kernels(kernel, M, N, K):
+    """Both quantizer kernels reduce the per-CTA maxima of the amax pass themselves and
+    publish g: g is the oracle's value bit for bit, and the output equals nvfp4_linear with
+    the separately computed scale."""
+    old = bsp.bsp_testing_set_quant_kernel(kernel)
+    try:
+        a_cpu = synth.bf16_normal((M, K), 1.0, 410 + M, 0.01, 20.0)
+        a = a_cpu.cuda()
+        w = synth.bf16_normal((N, K), 0.02, 411).cuda()
+        wc, wsf, gw = prepared_weight(w)
+        y, g = bsp.nvfp4_linear_dynamic(a, wc, wsf, gw)
+        ref = bsp.nvfp4_linear(a, bsp.nvfp4_global_scale(a), wc, wsf, gw)
+        torch.cuda.synchronize()
+        assert bsp.bsp_last_device_status() == 0
+        assert g.item() == float(oracle.nvfp4_global_scale(a_cpu))
+        assert torch.equal(y, ref)
+    finally:
+        bsp.bsp_testing_set_quant_kernel(old)
+
+
+@pytest.mark.parametrize("kernel", [1, 2])
+def test_linear_dynamic_all_zero_activations(kernel):
+    """amax = 0 gives g = 0: every activation code and block scale is zero, the product
+    vanishes (alpha = 0) and the output is the bias, exactly."""
+    old = bsp.bsp_testing_set_quant_kernel(kernel)
+    try:
+        M, N, K = 256, 384, 512
+        a = torch.zeros((M, K), dtype=torch.bfloat16, device="cuda")
+        w = synth.bf16_normal((N, K), 0.02, 420).cuda()
+        b = synth.bf16_normal((N,), 0.1, 421).cuda()
+        wc, wsf, gw = prepared_weight(w)
+        y, g = bsp.nvfp4_linear_dynamic(a, wc, wsf, gw, bias=b)
+        torch.cuda.synchronize()
+        assert bsp.bsp_last_device_status() == 0
+        assert g.item() == 0.0
+        assert torch.equal(y, b.expand(M, N))
+    finally:
+        bsp.bsp_testing_set_quant_kernel(old)
