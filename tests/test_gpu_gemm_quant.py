@@ -31,6 +31,9 @@ def prepared(x):
     (1, 64, 64, 2, False),           # one row, one 64-column group
     (384, 1024, 1280, 3, True),
     (4096, 12288, 3072, 4, False),   # the MLP up projection at 1 MP
+    (2560, 2112, 256, 5, True),      # 90 tiles for 74 CTA pairs: second tiles in the ragged
+                                     # last tile column, bias fetched ahead for them
+    (4096, 12288, 3072, 6, True),    # the MLP up projection with bias (768 tiles)
 ])
 def test_gemm_quant_equals_gemm_then_quantize(M, N, K, seed, with_bias):
     a = synth.bf16_normal((M, K), 1.0, seed, 0.005, 30.0).cuda()
