@@ -198,6 +198,30 @@ def cpu_oracle_sample(wl, rows: int, A=None, W=None):
     return dt, 2.0 * rows * wl.N * wl.K, oracle.default_threads()
 
 
+def cpu_quantize_one_thread(wl, rows: int, A=None) -> dict:
+    """The oracle's activation quantizer alone on one host thread, over `rows` rows of A
+    (the workload's scheme; its algorithmic bytes per element as the GPU kernel's)."""
+    import numpy as np
+    import oracle
+    import torch
+    A = wl.A() if A is None else A
+    rows = min(rows, A.shape[0])
+    idx = torch.from_numpy(np.linspace(0, A.shape[0] - 1, rows).astype(np.int64))
+    a_rows = A[idx].contiguous()
+    if wl.scheme == "nvfp4":
+        g = oracle.nvfp4_global_scale(A)
+        t0 = time.perf_counter()
+        oracle.nvfp4_quantize(a_rows, g, threads=1)
+        per_elt = 2.5625
+    else:
+        t0 = time.perf_counter()
+        oracle.fp8r_quantize(a_rows, threads=1)
+        per_elt = 2.0 + 1.0 + 4.0 / a_rows.shape[1]
+    dt = time.perf_counter() - t0
+    return {"value": rows * a_rows.shape[1] * per_elt / dt / 1e9, "unit": "GB/s", "threads": 1,
+            "rows": rows}
+
+
 def run_reference(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -473,7 +497,8 @@ def run_bsp(args):
             "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
             "sample": f"{min(args.cpu_rows, M)} of {M} rows of A: quantize + fp64 GEMM "
                       f"against the full weight ({dt:.1f} s)"
-                      + ("; first linear of the chain only" if args.chain else "")}
+                      + ("; first linear of the chain only" if args.chain else ""),
+            "quantize_one_thread": cpu_quantize_one_thread(wl, args.cpu_rows, A_cpu)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graphs, gs
