@@ -139,6 +139,31 @@ def _dtype(t, dt, what):
         raise TypeError(f"{what} must be {dt}, got {t.dtype}")
 
 
+def _buf(t, dt, what, min_numel: int):
+    """A buffer the library reads or writes `min_numel` elements of: dtype and size are
+    checked here, since the C calls receive only its address."""
+    if t is None:
+        return
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what} must be a torch.Tensor")
+    _dtype(t, dt, what)
+    if t.numel() < min_numel:
+        raise BSPError(f"argument check ({what} holds {t.numel()} elements, needs {min_numel})",
+                       -1)
+
+
+def _mat(t, dt, what, cols=None):
+    """A 2-D operand whose shape gives the problem size; returns (rows, cols)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{what} must be a torch.Tensor")
+    _dtype(t, dt, what)
+    if t.dim() != 2:
+        raise BSPError(f"argument check ({what} must be 2-D, got {tuple(t.shape)})", -1)
+    if cols is not None and t.shape[1] != cols:
+        raise BSPError(f"argument check ({what} has {t.shape[1]} columns, needs {cols})", -1)
+    return t.shape[0], t.shape[1]
+
+
 # ------------------------------------------------------------------ entry points
 def nvfp4_sf_bytes(rows: int, K: int, layout: int = SF_MMA) -> int:
     n = lib().nvfp4_sf_bytes(rows, K, layout)
@@ -150,29 +175,38 @@ def nvfp4_sf_bytes(rows: int, K: int, layout: int = SF_MMA) -> int:
 def nvfp4_quantize_act(x: torch.Tensor, global_scale: torch.Tensor, codes=None, scales=None,
                        layout: int = SF_MMA, stream=None):
     """bf16 [M, K] -> (codes uint8 [M, K/2], block scales uint8 in `layout`)."""
-    _dtype(x, torch.bfloat16, "x")
-    _dtype(global_scale, torch.float32, "global_scale")
-    M, K = x.shape
+    M, K = _mat(x, torch.bfloat16, "x")
+    _buf(global_scale, torch.float32, "global_scale", 1)
     if codes is None:
         codes = torch.empty((M, K // 2), dtype=torch.uint8, device=x.device)
     if scales is None:
         scales = torch.empty((max(nvfp4_sf_bytes(M, K, layout), 0),), dtype=torch.uint8,
                              device=x.device)
+    _buf(codes, torch.uint8, "codes", M * (K // 2))
+    _buf(scales, torch.uint8, "scales", max(nvfp4_sf_bytes(M, K, layout), 0))
     _check("nvfp4_quantize_act",
            lib().nvfp4_quantize_act(_ptr(x), M, K, _ptr(global_scale), _ptr(codes),
                                     _ptr(scales), layout, _stream(stream)))
     return codes, scales
 
 
+def _nvfp4_operands(M, N, K, a_sf, a_global, w_sf, w_global, bias):
+    _buf(a_sf, torch.uint8, "a_sf", max(nvfp4_sf_bytes(M, K, SF_MMA), 0))
+    _buf(a_global, torch.float32, "a_global", 1)
+    _buf(w_sf, torch.uint8, "w_sf", max(nvfp4_sf_bytes(N, K, SF_MMA), 0))
+    _buf(w_global, torch.float32, "w_global", 1)
+    _buf(bias, torch.bfloat16, "bias", N)
+
+
 def nvfp4_gemm(a_codes, a_sf, a_global, w_codes, w_sf, w_global, bias=None, out=None,
                stream=None):
     """Y[M, N] bf16 = (a_global*w_global) * (A_q . W_q^T) (+ bias); scales in SF_MMA layout."""
-    M, K2 = a_codes.shape
-    N = w_codes.shape[0]
-    if w_codes.shape[1] != K2:
-        raise BSPError("nvfp4_gemm (K mismatch)", -1)
+    M, K2 = _mat(a_codes, torch.uint8, "a_codes")
+    N, _ = _mat(w_codes, torch.uint8, "w_codes", K2)
+    _nvfp4_operands(M, N, 2 * K2, a_sf, a_global, w_sf, w_global, bias)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_codes.device)
+    _buf(out, torch.bfloat16, "out", M * N)
     _check("nvfp4_gemm",
            lib().nvfp4_gemm(_ptr(a_codes), _ptr(a_sf), _ptr(a_global), _ptr(w_codes),
                             _ptr(w_sf), _ptr(w_global), _ptr(bias), _ptr(out), M, N, 2 * K2,
@@ -184,15 +218,17 @@ def nvfp4_gemm_quant(a_codes, a_sf, a_global, w_codes, w_sf, w_global, out_globa
                      out_codes=None, out_sf=None, stream=None):
     """nvfp4_gemm whose bf16 output is re-quantized in the epilogue for the next nvfp4
     linear: returns (codes uint8 [M, N/2], MMA-layout scales) under `out_global`."""
-    M, K2 = a_codes.shape
-    N = w_codes.shape[0]
-    if w_codes.shape[1] != K2:
-        raise BSPError("nvfp4_gemm_quant (K mismatch)", -1)
+    M, K2 = _mat(a_codes, torch.uint8, "a_codes")
+    N, _ = _mat(w_codes, torch.uint8, "w_codes", K2)
+    _nvfp4_operands(M, N, 2 * K2, a_sf, a_global, w_sf, w_global, bias)
+    _buf(out_global, torch.float32, "out_global", 1)
     if out_codes is None:
         out_codes = torch.empty((M, N // 2), dtype=torch.uint8, device=a_codes.device)
     if out_sf is None:
         out_sf = torch.empty((max(nvfp4_sf_bytes(M, N, SF_MMA), 0),), dtype=torch.uint8,
                              device=a_codes.device)
+    _buf(out_codes, torch.uint8, "out_codes", M * (N // 2))
+    _buf(out_sf, torch.uint8, "out_sf", max(nvfp4_sf_bytes(M, N, SF_MMA), 0))
     _check("nvfp4_gemm_quant",
            lib().nvfp4_gemm_quant(_ptr(a_codes), _ptr(a_sf), _ptr(a_global), _ptr(w_codes),
                                   _ptr(w_sf), _ptr(w_global), _ptr(bias), _ptr(out_global),
@@ -212,17 +248,17 @@ def nvfp4_linear(x: torch.Tensor, input_scale: torch.Tensor, w_codes, w_sf, w_sc
     """Y[M, N] bf16 = nvfp4 linear of bf16 x [M, K]: activation quantizer + FP4 GEMM in one
     call (the GEMM overlaps the quantizer's tail).  `workspace` (uint8, at least
     nvfp4_linear_workspace_bytes(M, K) bytes) is allocated here when not given."""
-    _dtype(x, torch.bfloat16, "x")
-    _dtype(input_scale, torch.float32, "input_scale")
-    M, K = x.shape
-    N = w_codes.shape[0]
-    if w_codes.shape[1] * 2 != K:
-        raise BSPError("nvfp4_linear (K mismatch)", -1)
+    M, K = _mat(x, torch.bfloat16, "x")
+    _buf(input_scale, torch.float32, "input_scale", 1)
+    N, _ = _mat(w_codes, torch.uint8, "w_codes", K // 2)
+    _nvfp4_operands(0, N, K, None, None, w_sf, w_scale, bias)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _buf(out, torch.bfloat16, "out", M * N)
     if workspace is None:
         workspace = torch.empty((max(nvfp4_linear_workspace_bytes(M, K), 0),), dtype=torch.uint8,
                                 device=x.device)
+    _buf(workspace, torch.uint8, "workspace", 0)
     _check("nvfp4_linear",
            lib().nvfp4_linear(_ptr(x), _ptr(input_scale), _ptr(w_codes), _ptr(w_sf),
                               _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K, _ptr(workspace),
@@ -239,12 +275,12 @@ def nvfp4_linear_noalloc(x: torch.Tensor, input_scale: torch.Tensor, w_codes, w_
     """nvfp4_linear with the library's own per-device buffer as workspace; allocates
     nothing, so `out` ([M, N] bf16) must be given.  Calls that can run concurrently on
     one device race on that buffer (see include/bsp.h)."""
-    _dtype(x, torch.bfloat16, "x")
-    _dtype(input_scale, torch.float32, "input_scale")
+    M, K = _mat(x, torch.bfloat16, "x")
+    _buf(input_scale, torch.float32, "input_scale", 1)
+    N, _ = _mat(w_codes, torch.uint8, "w_codes", K // 2)
+    _nvfp4_operands(0, N, K, None, None, w_sf, w_scale, bias)
     _dtype(out, torch.bfloat16, "out")
-    M, K = x.shape
-    N = w_codes.shape[0]
-    if w_codes.shape[1] * 2 != K or tuple(out.shape) != (M, N):
+    if tuple(out.shape) != (M, N):
         raise BSPError("nvfp4_linear_noalloc (shape mismatch)", -1)
     _check("nvfp4_linear_noalloc",
            lib().nvfp4_linear_noalloc(_ptr(x), _ptr(input_scale), _ptr(w_codes), _ptr(w_sf),
@@ -257,18 +293,19 @@ def nvfp4_linear_dynamic(x: torch.Tensor, w_codes, w_sf, w_scale, bias=None, out
                          input_scale_out=None, workspace=None, stream=None):
     """nvfp4_linear with input_scale = amax(x) / (448*6) computed on the device for this
     call; returns (out, input_scale_out)."""
-    _dtype(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = w_codes.shape[0]
-    if w_codes.shape[1] * 2 != K:
-        raise BSPError("nvfp4_linear_dynamic (K mismatch)", -1)
+    M, K = _mat(x, torch.bfloat16, "x")
+    N, _ = _mat(w_codes, torch.uint8, "w_codes", K // 2)
+    _nvfp4_operands(0, N, K, None, None, w_sf, w_scale, bias)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _buf(out, torch.bfloat16, "out", M * N)
     if input_scale_out is None:
         input_scale_out = torch.empty((1,), dtype=torch.float32, device=x.device)
+    _buf(input_scale_out, torch.float32, "input_scale_out", 1)
     if workspace is None:
         workspace = torch.empty((max(nvfp4_linear_workspace_bytes(M, K), 0),), dtype=torch.uint8,
                                 device=x.device)
+    _buf(workspace, torch.uint8, "workspace", 0)
     _check("nvfp4_linear_dynamic",
            lib().nvfp4_linear_dynamic(_ptr(x), _ptr(input_scale_out), _ptr(w_codes), _ptr(w_sf),
                                       _ptr(w_scale), _ptr(bias), _ptr(out), M, N, K,
@@ -278,12 +315,13 @@ def nvfp4_linear_dynamic(x: torch.Tensor, w_codes, w_sf, w_scale, bias=None, out
 
 def fp8r_quantize_rows(x: torch.Tensor, q=None, row_scale=None, stream=None):
     """bf16 [M, K] -> (E4M3 codes uint8 [M, K], fp32 row scales [M])."""
-    _dtype(x, torch.bfloat16, "x")
-    M, K = x.shape
+    M, K = _mat(x, torch.bfloat16, "x")
     if q is None:
         q = torch.empty((M, K), dtype=torch.uint8, device=x.device)
     if row_scale is None:
         row_scale = torch.empty((M,), dtype=torch.float32, device=x.device)
+    _buf(q, torch.uint8, "q", M * K)
+    _buf(row_scale, torch.float32, "row_scale", M)
     _check("fp8r_quantize_rows",
            lib().fp8r_quantize_rows(_ptr(x), M, K, _ptr(q), _ptr(row_scale), _stream(stream)))
     return q, row_scale
@@ -301,16 +339,17 @@ def fp8r_linear(x: torch.Tensor, w_q, w_row_scale, bias=None, out=None, workspac
     """Y[M, N] bf16 = fp8r linear of bf16 x [M, K]: row quantizer + FP8 GEMM in one call.
     `workspace` (uint8, at least fp8r_linear_workspace_bytes(M, K) bytes) is allocated here
     when not given."""
-    _dtype(x, torch.bfloat16, "x")
-    M, K = x.shape
-    N = w_q.shape[0]
-    if w_q.shape[1] != K:
-        raise BSPError("fp8r_linear (K mismatch)", -1)
+    M, K = _mat(x, torch.bfloat16, "x")
+    N, _ = _mat(w_q, torch.uint8, "w_q", K)
+    _buf(w_row_scale, torch.float32, "w_row_scale", N)
+    _buf(bias, torch.bfloat16, "bias", N)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    _buf(out, torch.bfloat16, "out", M * N)
     if workspace is None:
         workspace = torch.empty((max(fp8r_linear_workspace_bytes(M, K), 0),),
                                 dtype=torch.uint8, device=x.device)
+    _buf(workspace, torch.uint8, "workspace", 0)
     _check("fp8r_linear",
            lib().fp8r_linear(_ptr(x), _ptr(w_q), _ptr(w_row_scale), _ptr(bias), _ptr(out), M, N, K,
                              _ptr(workspace), workspace.numel(), _stream(stream)))
@@ -319,12 +358,14 @@ def fp8r_linear(x: torch.Tensor, w_q, w_row_scale, bias=None, out=None, workspac
 
 def fp8r_gemm(a_q, a_row_scale, w_q, w_row_scale, bias=None, out=None, stream=None):
     """Y[M, N] bf16 = (A_q . W_q^T) * sA[m] * sW[n] (+ bias)."""
-    M, K = a_q.shape
-    N = w_q.shape[0]
-    if w_q.shape[1] != K:
-        raise BSPError("fp8r_gemm (K mismatch)", -1)
+    M, K = _mat(a_q, torch.uint8, "a_q")
+    N, _ = _mat(w_q, torch.uint8, "w_q", K)
+    _buf(a_row_scale, torch.float32, "a_row_scale", M)
+    _buf(w_row_scale, torch.float32, "w_row_scale", N)
+    _buf(bias, torch.bfloat16, "bias", N)
     if out is None:
         out = torch.empty((M, N), dtype=torch.bfloat16, device=a_q.device)
+    _buf(out, torch.bfloat16, "out", M * N)
     _check("fp8r_gemm",
            lib().fp8r_gemm(_ptr(a_q), _ptr(a_row_scale), _ptr(w_q), _ptr(w_row_scale),
                            _ptr(bias), _ptr(out), M, N, K, _stream(stream)))
@@ -336,6 +377,7 @@ def nvfp4_global_scale(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
     _dtype(x, torch.bfloat16, "x")
     if out is None:
         out = torch.empty((1,), dtype=torch.float32, device=x.device)
+    _buf(out, torch.float32, "out", 1)
     _check("nvfp4_global_scale",
            lib().nvfp4_global_scale(_ptr(x), x.numel(), _ptr(out), _stream(stream)))
     return out
@@ -343,9 +385,11 @@ def nvfp4_global_scale(x: torch.Tensor, out=None, stream=None) -> torch.Tensor:
 
 def nvfp4_sf_convert(src, rows: int, K: int, from_layout: int, to_layout: int, dst=None,
                      stream=None):
+    _buf(src, torch.uint8, "src", nvfp4_sf_bytes(rows, K, from_layout))
     if dst is None:
         dst = torch.empty((nvfp4_sf_bytes(rows, K, to_layout),), dtype=torch.uint8,
                           device=src.device)
+    _buf(dst, torch.uint8, "dst", nvfp4_sf_bytes(rows, K, to_layout))
     _check("nvfp4_sf_convert",
            lib().nvfp4_sf_convert(_ptr(src), _ptr(dst), rows, K, from_layout, to_layout,
                                   _stream(stream)))
@@ -356,10 +400,13 @@ def nvfp4_dequantize(codes: torch.Tensor, scales: torch.Tensor, global_scale: to
                      layout: int = SF_MMA, out=None, stream=None) -> torch.Tensor:
     """NVFP4 codes [rows, K/2] + block scales + fp32 global scale -> bf16 [rows, K]
     (the dequantise-only fallback's weight decode; see nvfp4_dequantize in bsp.h)."""
-    _dtype(codes, torch.uint8, "codes")
-    rows, K = codes.shape[0], 2 * codes.shape[1]
+    rows, K2 = _mat(codes, torch.uint8, "codes")
+    K = 2 * K2
+    _buf(scales, torch.uint8, "scales", max(nvfp4_sf_bytes(rows, K, layout), 0))
+    _buf(global_scale, torch.float32, "global_scale", 1)
     if out is None:
         out = torch.empty((rows, K), dtype=torch.bfloat16, device=codes.device)
+    _buf(out, torch.bfloat16, "out", rows * K)
     _check("nvfp4_dequantize",
            lib().nvfp4_dequantize(_ptr(codes), _ptr(scales), layout, _ptr(global_scale), rows, K,
                                   _ptr(out), _stream(stream)))

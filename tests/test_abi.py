@@ -197,6 +197,7 @@ def test_python_binding_refuses_cpu_tensors():
     import torch
     x = torch.zeros((128, 256), dtype=torch.bfloat16)
     g = torch.ones((1,), dtype=torch.float32)
-    with pytest.raises(bsp.BSPError):
-        bsp.nvfp4_quantize_act(x, g, codes=torch.empty(0, dtype=torch.uint8),
-                               scales=torch.empty(0, dtype=torch.uint8))
+    with pytest.raises(bsp.BSPError, match="not on a CUDA device"):
+        bsp.nvfp4_quantize_act(x, g, codes=torch.empty((128, 128), dtype=torch.uint8),
+                               scales=torch.empty((bsp.nvfp4_sf_bytes(128, 256),),
+                                                  dtype=torch.uint8))
