@@ -4,17 +4,28 @@ projection).
 
 "BFL (fp8r / nvfp4)" (Diffusers quantization doc), Kernels table: every nvfp4 linear
 quantizes its activations before the FP4 GEMM.  The fused epilogue must give exactly
-the codes and scale bytes of nvfp4_gemm followed by nvfp4_quantize_act on its bf16
-output (that two-call path is itself checked against the oracle in test_gpu_gemm.py,
-including the MLP chain), and the chained down projection must then match too.
+the codes and scale bytes that the oracle's NVFP4 quantizer gives on the GEMM's bf16
+output (oracle arm, every shape), and the same bytes as nvfp4_gemm followed by
+nvfp4_quantize_act; the chained down projection must then match too.
 """
 import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 import block_scaled_precision_act_b200 as bsp
 from parity import sf_valid_mask
+
+
+def assert_oracle_requantization(y, g_out, codes, sf, M, N):
+    """Codes and valid MMA-layout scale bytes of the fused epilogue equal the oracle's
+    quantizer run on the bf16 output y with the next layer's global scale g_out."""
+    c_or, s_lin = oracle.nvfp4_quantize(y.cpu(), np.float32(g_out.item()))
+    s_or = oracle.sf_linear_to_mma(s_lin, M, N)
+    valid = sf_valid_mask(M, N)
+    assert np.array_equal(codes.cpu().numpy(), c_or)
+    assert np.array_equal(sf.cpu().numpy()[valid], s_or[valid])
 
 pytestmark = pytest.mark.gpu
 
@@ -53,6 +64,7 @@ def test_gemm_quant_equals_gemm_then_quantize(M, N, K, seed, with_bias):
     assert torch.equal(codes, c_ref)
     valid = torch.from_numpy(sf_valid_mask(M, N)).cuda()
     assert torch.equal(sf[valid], s_ref[valid])
+    assert_oracle_requantization(y, g_out, codes, sf, M, N)
 
 
 def test_gemm_quant_with_saturating_scale():
@@ -72,6 +84,7 @@ def test_gemm_quant_with_saturating_scale():
     valid = torch.from_numpy(sf_valid_mask(M, N)).cuda()
     assert torch.equal(sf[valid], s_ref[valid])
     assert (s_ref[valid] == 0x7E).any()
+    assert_oracle_requantization(y, g_out, codes, sf, M, N)
 
 
 def test_mlp_chain_through_fused_requantization():
