@@ -114,6 +114,16 @@ def _check(fn: str, st: int) -> None:
         raise BSPError(fn, st)
 
 
+def _require_current_device(index: int, current: int | None = None) -> None:
+    """The C calls run on the current CUDA device and stream (cudaGetDevice): a tensor on
+    any other device would be handed to that device's kernels as a peer address, so it
+    is refused here."""
+    cur = torch.cuda.current_device() if current is None else current
+    if index != cur:
+        raise BSPError(f"argument check (tensor on cuda:{index}, but the current device is "
+                       f"cuda:{cur}; use torch.cuda.device)", -1)
+
+
 def _ptr(t):
     if t is None:
         return None
@@ -121,6 +131,7 @@ def _ptr(t):
         raise TypeError("expected a torch.Tensor")
     if not t.is_cuda:
         raise BSPError("argument check (tensor not on a CUDA device)", -1)
+    _require_current_device(t.device.index)
     if not t.is_contiguous():
         raise BSPError("argument check (tensor not contiguous)", -1)
     return t.data_ptr()

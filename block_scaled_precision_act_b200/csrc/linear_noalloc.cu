@@ -9,10 +9,16 @@
 // performs no allocation of any kind: no cudaMalloc, no cudaFree, no torch tensor.
 //
 // The buffer is g_linear_scratch below: kNoallocScratchBytes (128 MiB) per device, a
-// file-scope __device__ array.  Its device address is looked up with
-// cudaGetSymbolAddress on the first call made on each device and cached; that lookup
-// loads this file's module if it is not loaded yet, so make the first call on each
-// device outside any stream capture.  Problems whose workspace
+// file-scope __device__ array.  It occupies 128 MiB of device memory on every device
+// where this file's module is loaded, from the load until the context is destroyed,
+// whether or not this entry point is ever called there: with eager module loading
+// (CUDA_MODULE_LOADING=EAGER) the load happens when the library's context is created;
+// with lazy loading (the default) it happens at the first cudaGetSymbolAddress below.
+// Its device address is looked up with cudaGetSymbolAddress on the first successful
+// call made on each device and cached; that lookup may load the module, so make the
+// first call on each device outside any stream capture.  A lookup that fails (for
+// example inside a capture) is not cached: the call returns BSP_ERR_CUDA, the runtime
+// error it raised is cleared, and the next call tries again.  Problems whose workspace
 // (nvfp4_linear_workspace_bytes(M, K)) exceeds the buffer are rejected with
 // BSP_ERR_UNSUPPORTED_SHAPE.  Nothing in the buffer has to start at zero: every
 // byte the GEMM reads is written first by the quantizer of the same call.
@@ -21,6 +27,7 @@
 // can run at the same time (different streams, or different host threads on streams
 // that are not ordered) race on it and corrupt each other's results.  Calls on one
 // stream are ordered and safe.
+#include <atomic>
 #include <cstdint>
 #include <mutex>
 
@@ -34,9 +41,25 @@ constexpr int64_t kNoallocScratchBytes = int64_t{128} << 20;
 __device__ __align__(256) uint8_t g_linear_scratch[kNoallocScratchBytes];
 
 constexpr int kMaxDevices = 64;
-std::once_flag g_scratch_once[kMaxDevices];
-void* g_scratch_addr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::atomic<void*> g_scratch_addr[kMaxDevices];
+std::mutex g_scratch_mutex;
+
+// Device address of the current device's buffer (the caller made `dev` current), or
+// nullptr when the lookup failed; a failure leaves no pending runtime error behind.
+void* scratch_address(int dev)
+{
+    void* p = g_scratch_addr[dev].load(std::memory_order_acquire);
+    if (p != nullptr) return p;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    p = g_scratch_addr[dev].load(std::memory_order_relaxed);
+    if (p != nullptr) return p;
+    if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || p == nullptr) {
+        cudaGetLastError();
+        return nullptr;
+    }
+    g_scratch_addr[dev].store(p, std::memory_order_release);
+    return p;
+}
 
 }  // namespace
 }  // namespace bsp
@@ -60,12 +83,10 @@ int nvfp4_linear_noalloc(const void* x_bf16, const float* input_scale, const uin
     int st = check_device(&dev, nullptr);
     if (st != BSP_OK) return st;
     if (dev < 0 || dev >= kMaxDevices) return BSP_ERR_UNSUPPORTED_DEVICE;
-    std::call_once(g_scratch_once[dev], [dev] {
-        g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_addr[dev], g_linear_scratch);
-    });
-    if (g_scratch_err[dev] != cudaSuccess || g_scratch_addr[dev] == nullptr) return BSP_ERR_CUDA;
+    void* scratch = scratch_address(dev);
+    if (scratch == nullptr) return BSP_ERR_CUDA;
     return nvfp4_linear(x_bf16, input_scale, w_codes, w_sf, w_scale, bias_bf16, out_bf16, M, N,
-                        K, g_scratch_addr[dev], kNoallocScratchBytes, stream);
+                        K, scratch, kNoallocScratchBytes, stream);
 }
 
 }  // extern "C"

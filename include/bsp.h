@@ -17,10 +17,17 @@
  * row-scaled FP8 GEMM.  These entry points are that pair of calls for each scheme.
  *
  * Conventions for every call
- *   - All pointers are DEVICE pointers unless stated otherwise, owned by the caller;
- *     the library allocates nothing and keeps no per-call state.  Every tensor is
- *     contiguous row-major.  All work is enqueued asynchronously on `stream`
- *     (NULL = the legacy default stream); nothing synchronises the host.
+ *   - All pointers are DEVICE pointers unless stated otherwise, owned by the caller.
+ *     The library makes no allocation and keeps no per-call state: what one call
+ *     computes depends only on its arguments.  It does keep a little process-wide
+ *     state: per device, a status word written by kernels whose bounded wait ran out
+ *     (read and cleared by bsp_last_device_status), cached device properties and
+ *     kernel attributes, and nvfp4_linear_noalloc's fixed 128 MiB buffer and its cached
+ *     address; process-wide, the wait limit (bsp_set_wait_limit_ms) and the kernel
+ *     choices that the bsp_testing_set_* hooks of bsp_testing.h switch.  Every tensor
+ *     is contiguous row-major.  All work is enqueued asynchronously on `stream`
+ *     (NULL = the legacy default stream) of the CURRENT device; nothing synchronises
+ *     the host.
  *   - Tensor pointers must be 16-byte aligned (BSP_ERR_MISALIGNED otherwise).
  *   - Argument errors are detected on the host before any launch and returned as a
  *     negative bsp_status; nothing is enqueued in that case.  A zero-sized problem
@@ -194,8 +201,14 @@ int64_t nvfp4_linear_workspace_bytes(int64_t M, int64_t K);
  * Arguments and results: those of nvfp4_linear minus workspace / workspace_bytes;
  * results are bit-identical to nvfp4_linear.  The quantized activations go to one
  * buffer of nvfp4_linear_noalloc_max_bytes() bytes (128 MiB) per device, compiled
- * into the library (a file-scope __device__ array); its address is looked up on the
- * first call on each device, so make that first call outside any stream capture.
+ * into the library (a file-scope __device__ array).
+ * Footprint: the buffer takes 128 MiB of device memory on every device where its
+ * module is loaded, until the context is destroyed, even in a process that never
+ * calls this function: at context creation under CUDA_MODULE_LOADING=EAGER, or at
+ * the first call of this function on the device under lazy loading (the default).
+ * Its address is looked up on the first call on each device (which may load the
+ * module), so make that first call outside any stream capture; a lookup that fails
+ * returns BSP_ERR_CUDA, leaves no pending CUDA error, and is retried by the next call.
  * Nothing in it needs to start at zero (each call writes what it reads).
  * Errors: BSP_ERR_UNSUPPORTED_SHAPE when nvfp4_linear_workspace_bytes(M, K) exceeds
  * the buffer; otherwise as nvfp4_linear.

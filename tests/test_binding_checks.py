@@ -152,3 +152,15 @@ def test_helper_buffers():
         bsp.nvfp4_dequantize(codes, u8(16), f32(1), out=bf16(M, K))
     with pytest.raises(bsp.BSPError, match=TOO_SMALL):
         bsp.nvfp4_dequantize(codes, sf, f32(1), out=bf16(M, K - 16))
+
+
+def test_tensor_on_another_device_is_refused():
+    """The C calls launch on the current device (cudaGetDevice) and its stream; a tensor
+    of another GPU would reach that device's kernels as a peer address.  The binding
+    refuses it: pinned on the decision itself, with the current device given."""
+    bsp._require_current_device(0, current=0)
+    bsp._require_current_device(3, current=3)
+    with pytest.raises(bsp.BSPError, match="current device is cuda:0"):
+        bsp._require_current_device(1, current=0)
+    with pytest.raises(bsp.BSPError, match="tensor on cuda:0"):
+        bsp._require_current_device(0, current=2)

@@ -63,9 +63,68 @@ def test_noalloc_leaves_free_memory_unchanged():
 
 
 def test_noalloc_rejects_oversize_problem():
-    K = 3072
-    need_rows = bsp.nvfp4_linear_noalloc_max_bytes() // (K // 2) + 1
-    assert bsp.nvfp4_linear_workspace_bytes(need_rows, K) > bsp.nvfp4_linear_noalloc_max_bytes()
-    P = 1 << 20   # never dereferenced: the size check comes first
-    st = bsp.lib().nvfp4_linear_noalloc(P, P, P, P, P, None, P, need_rows, 256, K, None)
-    assert st == -2
+    """A problem whose workspace exceeds the fixed buffer is refused before any launch
+    (real buffers of the full size: no call here hands the library an address it does
+    not own)."""
+    K, N = 3072, 256
+    rows = bsp.nvfp4_linear_noalloc_max_bytes() // (K // 2) + 1
+    assert bsp.nvfp4_linear_workspace_bytes(rows, K) > bsp.nvfp4_linear_noalloc_max_bytes()
+    a = torch.zeros((rows, K), dtype=torch.bfloat16, device="cuda")
+    _, ga, wc, wsf, gw, _ = problem(128, N, K, 530, False)
+    y = torch.zeros((rows, N), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(bsp.BSPError) as err:
+        bsp.nvfp4_linear_noalloc(a, ga, wc, wsf, gw, out=y)
+    assert err.value.status == -2
+    torch.cuda.synchronize()
+    assert not torch.any(y)                              # nothing was launched
+    assert bsp.bsp_last_device_status() == 0
+
+
+CAPTURE_FIRST = r"""
+import sys, torch
+sys.path.insert(0, {root!r})
+sys.path.insert(0, {tests!r})
+import synth
+import block_scaled_precision_act_b200 as bsp
+a = synth.bf16_normal((256, 512), 1.0, 540).cuda()
+w = synth.bf16_normal((384, 512), 0.02, 541).cuda()
+ga, gw = bsp.nvfp4_global_scale(a), bsp.nvfp4_global_scale(w)
+wc, wsf = bsp.nvfp4_quantize_act(w, gw)
+ref = bsp.nvfp4_linear(a, ga, wc, wsf, gw)        # every other path initialised first
+torch.cuda.synchronize()
+y = torch.empty_like(ref)
+stream = torch.cuda.Stream()
+graph = torch.cuda.CUDAGraph()
+first = "captured"
+try:
+    with torch.cuda.graph(graph, stream=stream):
+        bsp.nvfp4_linear_noalloc(a, ga, wc, wsf, gw, out=y)
+except Exception as e:                            # the lookup may be refused in a capture
+    first = "refused: " + type(e).__name__
+torch.cuda.synchronize()
+del graph
+y2 = bsp.nvfp4_linear_noalloc(a, ga, wc, wsf, gw)  # retried outside the capture
+c, s = bsp.nvfp4_quantize_act(a, ga)              # no stale CUDA error left behind
+torch.cuda.synchronize()
+assert torch.equal(y2, ref), "noalloc after the capture differs from nvfp4_linear"
+assert bsp.bsp_last_device_status() == 0
+print("OK", first)
+"""
+
+
+def test_noalloc_first_call_inside_a_capture_does_not_poison_later_calls():
+    """The buffer's address is looked up on the first call on a device, which the header
+    asks callers to make outside stream capture.  If a caller makes it inside one and the
+    lookup is refused, that call fails, but the failure must not stay cached nor leave a
+    pending CUDA error: the next call outside the capture succeeds and equals
+    nvfp4_linear, and the next unrelated library call returns OK.  Run in a fresh
+    process, so that this really is the first call on the device."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = CAPTURE_FIRST.format(root=root, tests=os.path.join(root, "tests"))
+    r = subprocess.run([sys.executable, "-c", code], capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stdout[-2000:] + r.stderr[-4000:]
+    assert "OK" in r.stdout
