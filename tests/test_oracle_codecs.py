@@ -160,7 +160,15 @@ def test_e4m3_saturates_and_keeps_sign():
 
 
 # ------------------------------------------------------------------ scale layouts
-def test_sf_mma_offsets_hand_computed():
+def test_sf_mma_offsets_worked_examples_of_the_published_layout():
+    """Worked examples of the scale-factor layout the block-scaled tensor-core MMA reads,
+    as the cuBLAS documentation publishes it ("1D Block Scaling Factors Layout": the
+    scales of 128 rows x 4 blocks form one 512-byte tile; inside it row r, block c sits
+    at 16 * (r % 32) + 4 * (r // 32) + c; tiles are ordered along K first, then along
+    rows).  Each expected offset below is read off that description for one (row,
+    block) pair, not recomputed by the oracle's formula.  This is the CPU side only: the
+    layout is pinned on the GPU by the single-hot GEMM tests, where the tensor cores
+    themselves read it."""
     K = 256                      # 16 blocks of 16 -> 4 column tiles of 4
     assert oracle.sf_mma_offset(0, 0, K) == 0
     assert oracle.sf_mma_offset(0, 1, K) == 1
@@ -175,6 +183,8 @@ def test_sf_mma_offsets_hand_computed():
 
 @pytest.mark.parametrize("R,K", [(128, 64), (256, 256), (384, 3072 // 4), (200, 192)])
 def test_sf_mma_layout_is_injective_and_padded(R, K):
+    """Injectivity check: no two (row, block) pairs share a byte and every offset lies
+    inside the padded size."""
     nb = K // 16
     total = oracle.sf_bytes(R, K, True)
     assert total == ((R + 127) // 128) * ((nb + 3) // 4) * 512
