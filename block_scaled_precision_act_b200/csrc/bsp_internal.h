@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <utility>
 #include <cuda_runtime.h>
 
 #include "bsp.h"
@@ -38,6 +39,28 @@ constexpr int kDynamicPartials = 2048;
 // amax pass into `partials`, then the quantizer reducing them (MMA scale layout).
 int dynamic_quantize_front(const void* x_bf16, int64_t M, int64_t K, uint32_t* partials,
                            float* g_out, uint8_t* codes, uint8_t* scales, bsp_stream_t stream);
+
+// Launch `kernel`; with `pdl` the launch allows programmatic stream serialisation, so
+// the grid may start (prologue: barriers, TMEM, tensor-map prefetch, or just being
+// scheduled) while the preceding grid in the stream finishes.  Every kernel launched
+// this way executes griddep_wait() before its first read of an input or write of an
+// output.
+template <typename... Params, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
+                          cudaStream_t s, bool pdl, Args&&... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(block, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 

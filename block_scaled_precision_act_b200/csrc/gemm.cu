@@ -365,16 +365,19 @@ __global__ void __launch_bounds__(kThreads, 1)
 //   warp 0       TMA producer (both CTAs) into a ring of K-stages of 128 bytes per row;
 //   warp 1       TMEM allocation; in CTA 0 one thread issues the MMAs;
 //   warps 2..4   (CTA 0, nvfp4) scale-factor copies smem -> TMEM, one chunk kind per
-//                warp (A, B rows 0-127, B rows 128-255).  A tcgen05.cp costs about as
-//                much issue time as an MMA K-step, so issuing them from the MMA thread
-//                would serialise them with the MMAs; from other warps they overlap.
-//                The copies go into one of two TMEM scale buffers (stage parity).
+//                warp (A, B rows 0-127, B rows 128-255).  A tcgen05.cp issued by the MMA
+//                thread costs it ~48 cycles of issue, serialised with the MMAs; from
+//                warps on other sub-partitions the copies overlap the MMAs.  The copies
+//                go into a ring of three TMEM scale buffers: with two, the copy warps'
+//                handshake (wait for a buffer's release, copy, hand over) does not fit in
+//                the one stage of MMAs the ring leaves them, and a K-stage takes ~680
+//                cycles instead of ~550 (512 of MMA work).
 //   warps 5..12  epilogue, two warps per 32-lane TMEM quadrant, 32-column subtiles.
-// TMEM columns: accumulator 0 = [0, 256), accumulator 1 = [160, 416) (they share 96
-// columns), scale buffers at [416, 464) and [464, 512).  The epilogue drains the shared
-// columns first and then releases the accumulator, so the next tile's MMAs overlap the
-// rest of the epilogue.  Output goes through a 64-byte-swizzled smem slab per warp and
-// a TMA store.
+// TMEM columns: accumulator 0 = [0, 256), accumulator 1 = [112, 368) (they share 144
+// columns), scale buffers at [368, 416), [416, 464) and [464, 512).  The epilogue drains
+// the shared columns first and then releases the accumulator, so the next tile's MMAs
+// overlap the rest of the epilogue.  Output goes through a 64-byte-swizzled smem slab per
+// warp and a TMA store.
 template <bool NVF4>
 struct PairCfg {
     // A stage holds ATOMS K-atoms (128 rows x 128 bytes each) of A and of B.  NVFP4 keeps
@@ -402,15 +405,21 @@ struct PairCfg {
     static constexpr int BIAS_WARP = NVF4 ? 4 * 32 * 2 : 0;
     static constexpr int OFF_BIAS = OFF_EPI + EPI_WARPS * 2 * EPI_SLAB;
     static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_WARP;
-    static constexpr int NUM_BARS = 2 * STAGES + 4 + 4;
+    static constexpr int SF_NBUF = 3;                  // ring of TMEM scale buffers
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_NBUF + 4;
     static constexpr int SMEM_BYTES = 1024 + OFF_BAR + NUM_BARS * 8 + 16;
-    static constexpr int ACC_STRIDE = 160;
-    static constexpr int SF_COL0 = 416;                // two buffers of 48 columns
+    // accumulator 1 starts at ACC_STRIDE; FP8 keeps no scale buffers, so its accumulators
+    // share only 96 columns (3 subtiles), NVFP4's 144 (5 subtiles, the last partly)
+    static constexpr int ACC_STRIDE = NVF4 ? 112 : 160;
+    static constexpr int SHARED_SUBTILES = (256 - ACC_STRIDE + 31) / 32;
+    static constexpr int SF_COL0 = 368;                // three buffers of 48 columns
     static constexpr int SF_BUF = 48;                  // SFA 16 + SFB 32 per K-stage
     static constexpr uint32_t IDESC = NVF4 ? idesc_nvf4(256, 256) : idesc_e4m3(256, 256);
     static_assert(SMEM_BYTES <= 232448, "shared memory budget");
     static_assert(OFF_EPI % 1024 == 0, "epilogue slabs must be 1024-byte aligned");
-    static_assert(SF_COL0 + 2 * SF_BUF <= 512 && ACC_STRIDE + 256 <= SF_COL0, "TMEM budget");
+    static_assert(SF_COL0 + SF_NBUF * SF_BUF <= 512 && (!NVF4 || ACC_STRIDE + 256 <= SF_COL0) &&
+                      ACC_STRIDE + 256 <= 512, "TMEM budget");
+    static_assert(SHARED_SUBTILES >= 1 && SHARED_SUBTILES <= 6, "shared subtiles");
     static_assert(!NVF4 || ATOMS == 1, "scale copies are staged per atom");
 };
 
@@ -436,9 +445,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     uint8_t* sEpi = smem + C::OFF_EPI;
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
     uint64_t* empty = full + STAGES;
-    uint64_t* sf_full = empty + STAGES;     // [2]
-    uint64_t* sf_empty = sf_full + 2;       // [2]
-    uint64_t* acc_full = sf_empty + 2;
+    uint64_t* sf_full = empty + STAGES;     // [SF_NBUF]
+    uint64_t* sf_empty = sf_full + C::SF_NBUF;   // [SF_NBUF]
+    uint64_t* acc_full = sf_empty + C::SF_NBUF;
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* fin = acc_empty + 1;
     uint64_t* cp_fin = fin + 1;             // copy warps' last commits
@@ -462,8 +471,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             mbar_init(full + s, 1);
             mbar_init(empty + s, 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(sf_full + b, 3);      // one commit per copy warp
+        for (int b = 0; b < C::SF_NBUF; ++b) {
+            mbar_init(sf_full + b, 3);      // one arrive per copy warp
             mbar_init(sf_empty + b, 1);
         }
         mbar_init(acc_full, 1);
@@ -617,10 +626,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + s * C::A_BYTES));
                     const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * C::B_BYTES));
                     const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
-                    for (int k = 0; k < nk; ++k) {
+                    // K-step k lies in atom k/4 (ATOM bytes further on: ATOM/16 in the
+                    // descriptor's address field), 32 bytes (2) per step inside it
+                    auto issue = [&](int k) {
                         const uint32_t acc = (kt > 0 || k > 0) ? 1u : 0u;
-                        // K-step k lies in atom k/4 (ATOM bytes further on: ATOM/16 in the
-                        // descriptor's address field), 32 bytes (2) per step inside it
                         const uint64_t koff = static_cast<uint64_t>((k >> 2) * (C::ATOM >> 4) +
                                                                     2 * (k & 3));
                         if constexpr (NVF4)
@@ -628,6 +637,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                                           sf + 16 + k * 8, acc);
                         else
                             mma_f8f6f4_pair(d_tmem, adesc + koff, bdesc + koff, C::IDESC, acc);
+                    };
+                    // A full K-stage is issued from straight-line code: the same MMAs from a
+                    // loop with a run-time trip count cost the issuing thread ~50 cycles
+                    // more each, which the tensor pipe cannot hide (measured).  Only a
+                    // ragged last stage takes the loop.
+                    if (nk == C::K_STAGE / C::K_MMA) {
+#pragma unroll
+                        for (int k = 0; k < C::K_STAGE / C::K_MMA; ++k) issue(k);
+                    } else {
+                        for (int k = 0; k < nk; ++k) issue(k);
                     }
                     tc_commit_pair(empty + s, 0x1);
                     if constexpr (NVF4) tc_commit_pair(sf_empty + b, 0x1);
@@ -635,8 +654,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         s = 0;
                         ph ^= 1u;
                     }
-                    b ^= 1;
-                    bph ^= static_cast<uint32_t>(b == 0);
+                    if (++b == C::SF_NBUF) {
+                        b = 0;
+                        bph ^= 1u;
+                    }
                 }
                 if (!ok) break;
                 tc_commit_pair(acc_full, 0x3);
@@ -664,7 +685,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         tc_fence_after();
                         const int nk = min(4, K / 64 - 4 * kt);
                         const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
-                        for (int kb = 0; kb < nk; ++kb) {
+                        auto copy = [&](int kb) {
                             if (which == 0)
                                 tmem_cp_32x128b_x4_pair(
                                     sf + kb * 4,
@@ -674,6 +695,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                                     sf + 16 + kb * 8 + (which - 1) * 4,
                                     sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES +
                                                             (which - 1) * 2048 + kb * 512)));
+                        };
+                        // straight-line issue for a full stage, as for the MMAs
+                        if (nk == 4) {
+#pragma unroll
+                            for (int kb = 0; kb < 4; ++kb) copy(kb);
+                        } else {
+                            for (int kb = 0; kb < nk; ++kb) copy(kb);
                         }
                         // Hand the buffer over with a fence and a plain arrive, not a commit:
                         // the MMAs that read it are issued after this arrive and queue behind
@@ -685,8 +713,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                             s = 0;
                             ph ^= 1u;
                         }
-                        b ^= 1;
-                        bph ^= static_cast<uint32_t>(b == 0);
+                        if (++b == C::SF_NBUF) {
+                            b = 0;
+                            bph ^= 1u;
+                        }
                     }
                 }
                 tc_commit_pair(cp_fin, 0x1);     // lets the teardown wait for every copy
@@ -710,6 +740,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             qg = __ldg(args.q_global);
             qt = __fmul_rn(6.0f, qg);
         }
+        // Subtiles of 32 columns in processing order `ord` (this warp takes the ords of
+        // its half h: h, h+2, h+4, h+6).  The ones shared with the other accumulator come
+        // first: for NVFP4, columns 112..255 of accumulator 0 are its subtiles 3..7 and
+        // columns 0..143 of accumulator 1 its subtiles 0..4 (FP8: 5..7 and 0..2).
+        auto subtile_of = [](int ord, int sacc_) {
+            return sacc_ == 0 ? (ord + 8 - C::SHARED_SUBTILES) & 7 : ord;
+        };
         // NVFP4: this warp's bias columns of a tile, into its smem buffer (lane L: 4
         // columns of subtile L/8); done ahead of the accumulator wait so that the load
         // latency is not on the epilogue's path
@@ -717,7 +754,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             if constexpr (NVF4) {
                 if (args.bias == nullptr) return;
                 const int ord = 2 * (lane >> 3) + h;
-                const int j = (acc_it_ & 1) == 0 ? (ord + 5) & 7 : ord;
+                const int j = subtile_of(ord, acc_it_ & 1);
                 const int n = (tile_ / num_m) * 256 + j * 32 + (lane & 7) * 4;
                 uint2 v = make_uint2(0u, 0u);
                 if (n < N) v = __ldg(reinterpret_cast<const uint2*>(args.bias + n));
@@ -757,18 +794,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             const float sa = sa_next;
             const uint32_t tq = tbase + (static_cast<uint32_t>(q * 32) << 16) +
                                 static_cast<uint32_t>(sacc * C::ACC_STRIDE);
-            // Subtiles of 32 columns.  The 3 shared with the other accumulator (columns
-            // 160..255 of accumulator 0, 0..95 of accumulator 1) come first: this warp's
-            // share of them (two for half 0, one for half 1) is read from TMEM before
-            // anything else, then the accumulator is released to the MMA thread.
-            uint32_t pre[2][32];
-            const int npre = (h == 0) ? 2 : 1;
+            // The subtiles shared with the other accumulator come first: this warp's share
+            // of them (NVFP4: three for half 0, two for half 1; FP8: two and one) is read
+            // from TMEM before anything else, then the accumulator is released to the MMA
+            // thread.
+            uint32_t pre[3][32];
+            const int npre = (C::SHARED_SUBTILES + 1 - h) / 2;
 #pragma unroll
-            for (int idx = 0; idx < 2; ++idx) {
+            for (int idx = 0; idx < 3; ++idx) {
                 if (idx < npre) {
                     const int ord = 2 * idx + h;
-                    const int j = sacc == 0 ? (ord + 5) & 7 : ord;
-                    tmem_ld_x32(tq + j * 32, pre[idx]);
+                    tmem_ld_x32(tq + subtile_of(ord, sacc) * 32, pre[idx]);
                 }
             }
             tmem_ld_wait();
@@ -778,12 +814,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
 #pragma unroll
             for (int idx = 0; idx < 4; ++idx) {
                 const int ord = 2 * idx + h;                        // 0..7
-                const int j = sacc == 0 ? (ord + 5) & 7 : ord;
+                const int j = subtile_of(ord, sacc);
                 const int n0 = nt * 256 + j * 32;
                 uint32_t r[32];
                 if (idx < npre) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) r[i] = (idx == 0) ? pre[0][i] : pre[1][i];
+                    for (int i = 0; i < 32; ++i)
+                        r[i] = (idx == 0) ? pre[0][i] : (idx == 1) ? pre[1][i] : pre[2][i];
                 } else {
                     tmem_ld_x32(tq + j * 32, r);
                     tmem_ld_wait();
@@ -1005,27 +1042,6 @@ int make_map(CUtensorMap* m, const void* base, uint64_t row_bytes, uint64_t rows
 {
     return make_map_2d(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, base, row_bytes, rows, kBKB, box_rows,
                        CU_TENSOR_MAP_SWIZZLE_128B);
-}
-
-// Launch `kernel`; with `pdl` the launch allows programmatic stream serialisation, so
-// the grid may start (prologue: barriers, TMEM, tensor-map prefetch) while the
-// preceding grid in the stream finishes.  The kernels' producers call griddep_wait()
-// before their first load.
-template <typename... Params, typename... Args>
-cudaError_t launch_kernel(void (*kernel)(Params...), unsigned grid, unsigned block, size_t smem,
-                          cudaStream_t s, bool pdl, Args&&... args)
-{
-    cudaLaunchConfig_t cfg = {};
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.gridDim = dim3(grid, 1, 1);
-    cfg.blockDim = dim3(block, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 template <bool NVF4, bool QOUT = false>
