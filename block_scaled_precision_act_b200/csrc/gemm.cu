@@ -684,24 +684,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         }
                         tc_fence_after();
                         const int nk = min(4, K / 64 - 4 * kt);
+                        // this warp's chunk kind: destination column and source descriptor of
+                        // its first 512-byte chunk; chunk kb is 512 bytes (32 in the
+                        // descriptor's 16-byte address field) further on in shared memory
+                        // and `dstep` columns further on in TMEM
                         const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
-                        auto copy = [&](int kb) {
-                            if (which == 0)
-                                tmem_cp_32x128b_x4_pair(
-                                    sf + kb * 4,
-                                    sdesc_sf_block(smem_u32(sSFA + s * C::SFA_BYTES + kb * 512)));
-                            else
-                                tmem_cp_32x128b_x4_pair(
-                                    sf + 16 + kb * 8 + (which - 1) * 4,
-                                    sdesc_sf_block(smem_u32(sSFB + s * C::SFB_BYTES +
-                                                            (which - 1) * 2048 + kb * 512)));
-                        };
-                        // straight-line issue for a full stage, as for the MMAs
+                        const uint32_t dst0 = which == 0 ? sf : sf + 16 + (which - 1) * 4;
+                        const uint32_t dstep = which == 0 ? 4u : 8u;
+                        const uint64_t src0 = sdesc_sf_block(smem_u32(
+                            which == 0 ? sSFA + s * C::SFA_BYTES
+                                       : sSFB + s * C::SFB_BYTES + (which - 1) * 2048));
+                        // straight-line issue for a full stage, as for the MMAs: a run-time
+                        // choice or trip count between the copies slows their issue
                         if (nk == 4) {
 #pragma unroll
-                            for (int kb = 0; kb < 4; ++kb) copy(kb);
+                            for (int kb = 0; kb < 4; ++kb)
+                                tmem_cp_32x128b_x4_pair(dst0 + kb * dstep, src0 + 32 * kb);
                         } else {
-                            for (int kb = 0; kb < nk; ++kb) copy(kb);
+                            for (int kb = 0; kb < nk; ++kb)
+                                tmem_cp_32x128b_x4_pair(dst0 + kb * dstep, src0 + 32 * kb);
                         }
                         // Hand the buffer over with a fence and a plain arrive, not a commit:
                         // the MMAs that read it are issued after this arrive and queue behind
