@@ -596,11 +596,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             int acc_it = 0;
             bool ok = true;
             for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
-                if (acc_it > 0 &&
-                    !mbar_wait(acc_empty, static_cast<uint32_t>((acc_it - 1) & 1), abort_flag,
-                               args.wait_ns, args.status, 12))
-                    break;
-                tc_fence_after();
                 const uint32_t d_tmem = tbase + static_cast<uint32_t>((acc_it & 1) * C::ACC_STRIDE);
                 for (int kt = 0; kt < num_kt; ++kt) {
                     // NVFP4: the copy warps hand over a stage's scales only after they have
@@ -611,18 +606,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         ok = false;
                         break;
                     }
-                    int nk;
-                    if constexpr (NVF4) {
-                        if (!mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status,
-                                       15)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        nk = min(4, K / 64 - 4 * kt);
-                    } else {
-                        nk = min(4 * C::ATOMS, (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
+                    if (NVF4 &&
+                        !mbar_wait(sf_full + b, bph, abort_flag, args.wait_ns, args.status, 15)) {
+                        ok = false;
+                        break;
                     }
+                    // A tile's first stage also needs its accumulator back from the epilogue.
+                    // Waited for after the stage's operands, which are normally ready long
+                    // before: the epilogue's release is the last event of the tile handoff.
+                    if (kt == 0 && acc_it > 0 &&
+                        !mbar_wait(acc_empty, static_cast<uint32_t>((acc_it - 1) & 1), abort_flag,
+                                   args.wait_ns, args.status, 12)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const int nk = NVF4 ? min(4, K / 64 - 4 * kt)
+                                        : min(4 * C::ATOMS,
+                                              (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
                     const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + s * C::A_BYTES));
                     const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * C::B_BYTES));
                     const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
@@ -826,9 +827,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     tmem_ld_x32(tq + j * 32, r);
                     tmem_ld_wait();
                 }
+                // a slab this warp may write: the TMA store that last read it must be done
+                // reading it
+                auto slab_ready = [&]() -> uint8_t* {
+                    if (lane == 0 && last_group[buf] >= 0) {
+                        if (committed - 1 - last_group[buf] == 0)
+                            bulk_wait_group_read<0>();
+                        else
+                            bulk_wait_group_read<1>();
+                    }
+                    __syncwarp();
+                    return slab0 + buf * C::EPI_SLAB;
+                };
                 uint32_t packed[16];
-                if (NVF4 && n0 + 32 <= N) {
-                    // whole subtile inside N: the four bias reads go out before the math
+                uint8_t* slab = nullptr;
+                if (NVF4 && !QOUT && n0 + 32 <= N) {
+                    // whole subtile inside N, bf16 out: each 8-column chunk goes to the slab
+                    // as soon as it is computed, so that few registers are live beside the
+                    // pre-read subtiles
+                    slab = slab_ready();
+                    const bool has_bias = args.bias != nullptr;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        float v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            v[i] = __fmul_rn(__uint_as_float(r[g * 8 + i]), alpha);
+                        if (has_bias) {
+                            const uint4 bb =
+                                *reinterpret_cast<const uint4*>(bias_w + idx * 64 + g * 16);
+                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                            for (int i = 0; i < 4; ++i) {
+                                v[2 * i] = __fadd_rn(v[2 * i], bf16lo_to_f32(bw[i]));
+                                v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16hi_to_f32(bw[i]));
+                            }
+                        }
+                        const int pc = g ^ ((lane >> 1) & 3);           // 64-byte swizzle
+                        *reinterpret_cast<uint4*>(slab + lane * 64 + pc * 16) =
+                            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                       pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                    }
+                } else if (NVF4 && n0 + 32 <= N) {
+                    // whole subtile inside N, re-quantized output (which needs all 32 values
+                    // in registers): the four bias reads go out before the math
                     uint4 bb[4];
                     const bool has_bias = args.bias != nullptr;
                     if (has_bias) {
@@ -854,41 +896,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                         for (int i = 0; i < 4; ++i)
                             packed[g * 4 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
                     }
-                } else
+                } else {
 #pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    const int n = n0 + g * 8;
-                    float v[8];
+                    for (int g = 0; g < 4; ++g) {
+                        const int n = n0 + g * 8;
+                        float v[8];
 #pragma unroll
-                    for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[g * 8 + i]);
-                    if (n < N) {
-                        if constexpr (NVF4) {
+                        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[g * 8 + i]);
+                        if (n < N) {
+                            if constexpr (NVF4) {
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], alpha);
-                        } else {
-                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(args.w_scale + n));
-                            const float4 w1 =
-                                __ldg(reinterpret_cast<const float4*>(args.w_scale + n + 4));
-                            const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+                                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(v[i], alpha);
+                            } else {
+                                const float4 w0 = __ldg(reinterpret_cast<const float4*>(args.w_scale + n));
+                                const float4 w1 =
+                                    __ldg(reinterpret_cast<const float4*>(args.w_scale + n + 4));
+                                const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], sa), sw[i]);
-                        }
-                        if (args.bias != nullptr) {
-                            uint4 bb;
-                            if constexpr (NVF4)
-                                bb = *reinterpret_cast<const uint4*>(bias_w + idx * 64 + g * 16);
-                            else
-                                bb = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
-                            const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+                                for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], sa), sw[i]);
+                            }
+                            if (args.bias != nullptr) {
+                                uint4 bb;
+                                if constexpr (NVF4)
+                                    bb = *reinterpret_cast<const uint4*>(bias_w + idx * 64 + g * 16);
+                                else
+                                    bb = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
+                                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                v[2 * i] = __fadd_rn(v[2 * i], bf16lo_to_f32(bw[i]));
-                                v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16hi_to_f32(bw[i]));
+                                for (int i = 0; i < 4; ++i) {
+                                    v[2 * i] = __fadd_rn(v[2 * i], bf16lo_to_f32(bw[i]));
+                                    v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16hi_to_f32(bw[i]));
+                                }
                             }
                         }
-                    }
 #pragma unroll
-                    for (int i = 0; i < 4; ++i) packed[g * 4 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                        for (int i = 0; i < 4; ++i) packed[g * 4 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+                    }
                 }
                 if constexpr (QOUT) {
                     // bf16(Y) re-quantized in registers: this lane's 32 columns are two
@@ -909,21 +952,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     }
                     continue;
                 }
-                // the TMA store that last read this slab must be done reading it
-                if (lane == 0 && last_group[buf] >= 0) {
-                    if (committed - 1 - last_group[buf] == 0)
-                        bulk_wait_group_read<0>();
-                    else
-                        bulk_wait_group_read<1>();
-                }
-                __syncwarp();
-                uint8_t* slab = slab0 + buf * C::EPI_SLAB;
+                if (slab == nullptr) {
+                    slab = slab_ready();
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const int pc = c ^ ((lane >> 1) & 3);           // 64-byte swizzle
-                    *reinterpret_cast<uint4*>(slab + lane * 64 + pc * 16) =
-                        make_uint4(packed[c * 4], packed[c * 4 + 1], packed[c * 4 + 2],
-                                   packed[c * 4 + 3]);
+                    for (int c = 0; c < 4; ++c) {
+                        const int pc = c ^ ((lane >> 1) & 3);           // 64-byte swizzle
+                        *reinterpret_cast<uint4*>(slab + lane * 64 + pc * 16) =
+                            make_uint4(packed[c * 4], packed[c * 4 + 1], packed[c * 4 + 2],
+                                       packed[c * 4 + 3]);
+                    }
                 }
                 fence_proxy_async_smem();
                 __syncwarp();
