@@ -595,6 +595,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             uint32_t bph = 0;
             int acc_it = 0;
             bool ok = true;
+            // descriptors of ring slot 0; slot s starts s * A_BYTES further on, A_BYTES / 16
+            // in the 16-byte address field (no carry: shared memory is below 256 KB)
+            const uint64_t adesc0 = sdesc_kmajor_sw128(smem_u32(sA));
+            const uint64_t bdesc0 = sdesc_kmajor_sw128(smem_u32(sB));
             for (int tile = pair; ok && tile < num_tiles; tile += npairs) {
                 const uint32_t d_tmem = tbase + static_cast<uint32_t>((acc_it & 1) * C::ACC_STRIDE);
                 for (int kt = 0; kt < num_kt; ++kt) {
@@ -624,8 +628,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                     const int nk = NVF4 ? min(4, K / 64 - 4 * kt)
                                         : min(4 * C::ATOMS,
                                               (K - kt * C::K_STAGE + C::K_MMA - 1) / C::K_MMA);
-                    const uint64_t adesc = sdesc_kmajor_sw128(smem_u32(sA + s * C::A_BYTES));
-                    const uint64_t bdesc = sdesc_kmajor_sw128(smem_u32(sB + s * C::B_BYTES));
+                    const uint64_t adesc = adesc0 + static_cast<uint64_t>(s * (C::A_BYTES >> 4));
+                    const uint64_t bdesc = bdesc0 + static_cast<uint64_t>(s * (C::B_BYTES >> 4));
                     const uint32_t sf = tbase + C::SF_COL0 + b * C::SF_BUF;
                     // K-step k lies in atom k/4 (ATOM bytes further on: ATOM/16 in the
                     // descriptor's address field), 32 bytes (2) per step inside it
