@@ -168,17 +168,19 @@ __global__ void __launch_bounds__(kQuantThreads)
     // a GEMM launched as this grid's programmatic dependent may start its prologue now;
     // it still waits for this grid to complete before reading the codes
     griddep_launch_dependents();
-    const float g = resolve_global_scale(gptr, partials, npartials, gout);
-    const float t = __fmul_rn(6.0f, g);
     const int lane = threadIdx.x & 31;
     const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x) >> 5;
     const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * kQuantThreads) >> 5;
     const int64_t kb4 = (nb_row + 3) >> 2;
     const int64_t step = nwarps * kQBlocksPerWarp;
 
+    // the first span's loads go out before the global scale is read (or reduced), so
+    // their latency and that of g overlap instead of adding up
     int64_t base = warp * kQBlocksPerWarp;
     Block16 b0 = load_block(x, base + lane, nblk);
     Block16 b1 = load_block(x, base + 32 + lane, nblk);
+    const float g = resolve_global_scale(gptr, partials, npartials, gout);
+    const float t = __fmul_rn(6.0f, g);
     while (base < nblk) {
         const int64_t next = base + step;
         // prefetch the next span before encoding this one
