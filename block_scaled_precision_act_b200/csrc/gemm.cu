@@ -373,6 +373,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 //                the one stage of MMAs the ring leaves them, and a K-stage takes ~680
 //                cycles instead of ~550 (512 of MMA work).
 //   warps 5..12  epilogue, two warps per 32-lane TMEM quadrant, 32-column subtiles.
+//                FP8: on a pair's last tile warps 0-3 take two subtiles per quadrant.
 // TMEM columns: accumulator 0 = [0, 256), accumulator 1 = [112, 368) (they share 144
 // columns), scale buffers at [368, 416), [416, 464) and [464, 512).  The epilogue drains
 // the shared columns first and then releases the accumulator, so the next tile's MMAs
@@ -406,7 +407,9 @@ struct PairCfg {
     static constexpr int OFF_BIAS = OFF_EPI + EPI_WARPS * 2 * EPI_SLAB;
     static constexpr int OFF_BAR = OFF_BIAS + EPI_WARPS * BIAS_WARP;
     static constexpr int SF_NBUF = 3;                  // ring of TMEM scale buffers
-    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_NBUF + 4;
+    // FP8: warps 0-3 help with the last tile's epilogue (see the kernel's tail)
+    static constexpr bool TAIL_HELP = !NVF4;
+    static constexpr int NUM_BARS = 2 * STAGES + 2 * SF_NBUF + 5;
     static constexpr int SMEM_BYTES = 1024 + OFF_BAR + NUM_BARS * 8 + 16;
     // accumulator 1 starts at ACC_STRIDE; FP8 keeps no scale buffers, so its accumulators
     // share only 96 columns (3 subtiles), NVFP4's 144 (5 subtiles, the last partly)
@@ -451,7 +454,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
     uint64_t* acc_empty = acc_full + 1;
     uint64_t* fin = acc_empty + 1;
     uint64_t* cp_fin = fin + 1;             // copy warps' last commits
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(cp_fin + 1);
+    uint64_t* help_go = cp_fin + 1;         // the pair's last tile is issued (see the tail)
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(help_go + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -479,6 +483,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         mbar_init(acc_empty, 2 * C::EPI_WARPS);   // epilogue warps of both CTAs
         mbar_init(fin, 1);
         mbar_init(cp_fin, 3);
+        mbar_init(help_go, 1);
         *abort_flag = 0;
         fence_mbar_init();
         prefetch_tmap(&tmA);
@@ -668,6 +673,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
                 tc_commit_pair(acc_full, 0x3);
                 ++acc_it;
             }
+            // every tile of the pair is issued (or the pair gave up): the helpers of the
+            // last tile's epilogue may now wait for its accumulator
+            if (C::TAIL_HELP && pair < num_tiles) {
+                mbar_arrive(help_go);
+                mbar_arrive_cluster_relaxed(mapa_shared(smem_u32(help_go), 1));
+            }
         }
     } else if (warp <= 4) {
         // ------------------------------------------------------------ scale copies (CTA 0)
@@ -817,8 +828,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster_relaxed(acc_empty0);   // values are in registers
+            // the pair's last tile: orders 6 and 7 go to the tail helpers (below)
+            const bool help_tail = C::TAIL_HELP && tile + npairs >= num_tiles;
 #pragma unroll
             for (int idx = 0; idx < 4; ++idx) {
+                if (idx == 3 && help_tail) continue;
                 const int ord = 2 * idx + h;                        // 0..7
                 const int j = subtile_of(ord, sacc);
                 const int n0 = nt * 256 + j * 32;
@@ -987,6 +1001,91 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         // the stores must have read their smem slabs before the CTA exits
         if (lane == 0) bulk_wait_group_read<0>();
         __syncwarp();
+    }
+
+    // ---------------------------------------------------------------- last-tile helpers
+    // FP8 (TAIL_HELP): on the pair's last tile the producer and MMA warps and warps 2-3
+    // (one per TMEM lane quadrant, idle by then in both CTAs) take the last two subtiles of
+    // their quadrant (orders 6 and 7), so each epilogue warp processes three subtiles there
+    // instead of four: that epilogue overlaps nothing, and FP8's second warp of a quadrant
+    // loads three of its four subtiles after the release (fp8r at 256 x 3072 x 3072:
+    // 17.0 -> 15.7 us; the NVFP4 kernel, whose two warps per quadrant are balanced, gained
+    // nothing from it).  Their slabs are in the operand ring, which the
+    // last tile's completed MMAs no longer read.  They wait on help_go first, which
+    // completes once every tile of the pair is issued, so the accumulator phase they then
+    // wait for cannot belong to an earlier tile of the same parity.  The arithmetic is the
+    // epilogue's generic path (bit-identical outputs).
+    if constexpr (C::TAIL_HELP) {
+        if (warp < 4 && pair < num_tiles) {
+            const int acc_last = (num_tiles - 1 - pair) / npairs;
+            const int last_tile = pair + acc_last * npairs;
+            __syncwarp();
+            const bool hok =
+                mbar_wait(help_go, 0, abort_flag, args.wait_ns, args.status, 18) &&
+                mbar_wait(acc_full, static_cast<uint32_t>(acc_last & 1), abort_flag,
+                          args.wait_ns, args.status, 19);
+            if (__all_sync(0xffffffffu, hok)) {
+                tc_fence_after();
+                // scales and bias may come from the preceding grid
+                griddep_wait();
+                const int q = warp;
+                const int mt = last_tile % num_m, nt = last_tile / num_m;
+                const int wrow = mt * 256 + static_cast<int>(rank) * 128 + q * 32;
+                const int m = wrow + lane;
+                const int sacc = acc_last & 1;
+                const uint32_t tq = tbase + (static_cast<uint32_t>(q * 32) << 16) +
+                                    static_cast<uint32_t>(sacc * C::ACC_STRIDE);
+                const float sa = m < M ? __ldg(args.a_scale + m) : 0.0f;   // row scale
+                const uint64_t policy = l2_policy_evict_first();
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const int ord = 6 + u;
+                    const int j = sacc == 0 ? (ord + 8 - C::SHARED_SUBTILES) & 7 : ord;
+                    const int n0 = nt * 256 + j * 32;
+                    uint32_t r[32];
+                    tmem_ld_x32(tq + j * 32, r);
+                    tmem_ld_wait();
+                    uint8_t* slab = sA + (warp * 2 + u) * C::EPI_SLAB;
+#pragma unroll
+                    for (int g = 0; g < 4; ++g) {
+                        const int n = n0 + g * 8;
+                        float v[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[g * 8 + i]);
+                        if (n < N) {
+                            const float4 w0 = __ldg(reinterpret_cast<const float4*>(args.w_scale + n));
+                            const float4 w1 =
+                                __ldg(reinterpret_cast<const float4*>(args.w_scale + n + 4));
+                            const float sw[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__fmul_rn(v[i], sa), sw[i]);
+                            if (args.bias != nullptr) {
+                                const uint4 bb = __ldg(reinterpret_cast<const uint4*>(args.bias + n));
+                                const uint32_t bw[4] = {bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    v[2 * i] = __fadd_rn(v[2 * i], bf16lo_to_f32(bw[i]));
+                                    v[2 * i + 1] = __fadd_rn(v[2 * i + 1], bf16hi_to_f32(bw[i]));
+                                }
+                            }
+                        }
+                        const int pc = g ^ ((lane >> 1) & 3);           // 64-byte swizzle
+                        *reinterpret_cast<uint4*>(slab + lane * 64 + pc * 16) =
+                            make_uint4(pack_bf16x2(v[0], v[1]), pack_bf16x2(v[2], v[3]),
+                                       pack_bf16x2(v[4], v[5]), pack_bf16x2(v[6], v[7]));
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (wrow < M && n0 < N && lane == 0) {
+                        tma_store_2d_hint(&tmY, slab, n0, wrow, policy);
+                        bulk_commit_group();
+                    }
+                }
+                // the stores must have read their slabs before the CTA exits
+                if (lane == 0) bulk_wait_group_read<0>();
+                __syncwarp();
+            }
+        }
     }
 
     // ---------------------------------------------------------------- teardown
