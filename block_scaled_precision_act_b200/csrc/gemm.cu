@@ -1019,9 +1019,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<NVF4>::THREA
         if (warp < 4 && pair < num_tiles) {
             const int acc_last = (num_tiles - 1 - pair) / npairs;
             const int last_tile = pair + acc_last * npairs;
+            // help_go spans the whole GEMM, not one stage or tile, so the per-wait limit
+            // (which may be set short) would misfire on long GEMMs; the MMA thread arrives
+            // on it even when it gives up, so a 60-second bound is only a safety net
+            const uint64_t go_ns = args.wait_ns > 60000000000ull ? args.wait_ns : 60000000000ull;
             __syncwarp();
             const bool hok =
-                mbar_wait(help_go, 0, abort_flag, args.wait_ns, args.status, 18) &&
+                mbar_wait(help_go, 0, abort_flag, go_ns, args.status, 18) &&
                 mbar_wait(acc_full, static_cast<uint32_t>(acc_last & 1), abort_flag,
                           args.wait_ns, args.status, 19);
             if (__all_sync(0xffffffffu, hok)) {

@@ -320,7 +320,10 @@ int64_t nvfp4_sf_bytes(int64_t rows, int64_t K, int layout);
 int bsp_last_device_status(bsp_stream_t stream);
 
 /* Bounded-wait limit of the GEMM kernels in milliseconds (default 2000, also set by
- * the BSP_WAIT_LIMIT_MS environment variable at first use).  Returns the old value. */
+ * the BSP_WAIT_LIMIT_MS environment variable at first use): the longest any one wait on a
+ * pipeline stage or tile may take.  (The fp8r kernel's last-tile helpers wait once for the
+ * whole GEMM's issue; that wait is bounded by the larger of this limit and 60 s.)  Returns
+ * the old value. */
 int64_t bsp_set_wait_limit_ms(int64_t ms);
 
 /* Human-readable name of a bsp_status value. */
