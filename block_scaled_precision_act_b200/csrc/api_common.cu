@@ -10,7 +10,7 @@ namespace {
 // Written by kernels when a bounded wait runs out: {status code, wait site}.
 __device__ int g_bsp_status[2];
 
-constexpr int kMaxDevices = 64;
+using bsp::kMaxDevices;
 std::once_flag g_dev_once[kMaxDevices];
 int g_dev_ok[kMaxDevices];
 int g_dev_sms[kMaxDevices];

@@ -9,6 +9,10 @@
 
 namespace bsp {
 
+// Devices the library keeps per-device state for (ids 0 .. kMaxDevices - 1; check_device
+// refuses others before any of that state is touched).
+constexpr int kMaxDevices = 64;
+
 // Returns BSP_OK when the current device is compute capability 10.0; caches per device.
 int check_device(int* device_out, int* num_sms_out);
 

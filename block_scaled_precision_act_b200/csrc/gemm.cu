@@ -1194,12 +1194,13 @@ int launch_pair(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int de
                 cudaStream_t s, bool pdl)
 {
     using C = PairCfg<NVF4>;
-    static std::once_flag once[64];
-    static cudaError_t err[64];
-    static int max_pairs[64];
+    static std::once_flag once[kMaxDevices];
+    static cudaError_t err[kMaxDevices];
+    static int max_pairs[kMaxDevices];
     std::call_once(once[dev], [&] {
         err[dev] = cudaFuncSetAttribute(gemm_pair_kernel<NVF4, QOUT>,
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+        if (err[dev] != cudaSuccess) cudaGetLastError();        // no stale error left behind
         max_pairs[dev] = sms / 2;
         if (err[dev] == cudaSuccess) {
             cudaLaunchConfig_t cfg = {};
@@ -1287,12 +1288,13 @@ int launch(const uint8_t* a, const uint8_t* w, const GemmArgs& args, int dev, in
            cudaStream_t s, bool pdl)
 {
     using C = Cfg<NVF4, BN, STAGES, NACC>;
-    static std::once_flag attr_once[64];
-    static cudaError_t attr_err[64];
+    static std::once_flag attr_once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
     std::call_once(attr_once[dev], [&] {
         attr_err[dev] = cudaFuncSetAttribute(gemm_kernel<NVF4, BN, STAGES, NACC>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              C::SMEM_BYTES);
+        if (attr_err[dev] != cudaSuccess) cudaGetLastError();   // no stale error left behind
     });
     if (attr_err[dev] != cudaSuccess) return BSP_ERR_CUDA;
     const uint64_t row_bytes = NVF4 ? static_cast<uint64_t>(args.K) / 2 : args.K;

@@ -40,7 +40,6 @@ constexpr int64_t kNoallocScratchBytes = int64_t{128} << 20;
 
 __device__ __align__(256) uint8_t g_linear_scratch[kNoallocScratchBytes];
 
-constexpr int kMaxDevices = 64;
 std::atomic<void*> g_scratch_addr[kMaxDevices];
 std::mutex g_scratch_mutex;
 

@@ -609,8 +609,8 @@ int quantize_act_impl(const void* x_bf16, int64_t M, int64_t K, const float* glo
         return launch_status();
     }
     // one persistent CTA per SM, each a contiguous range of whole 64-block warp spans
-    static std::once_flag attr_once[64];
-    static cudaError_t attr_err[64];
+    static std::once_flag attr_once[kMaxDevices];
+    static cudaError_t attr_err[kMaxDevices];
     std::call_once(attr_once[dev], [dev] {
         cudaError_t e = cudaSuccess;
         for (auto k : {nvfp4_quant_staged_kernel<BSP_SF_LINEAR, false>,
@@ -618,6 +618,7 @@ int quantize_act_impl(const void* x_bf16, int64_t M, int64_t K, const float* glo
                        nvfp4_quant_staged_kernel<BSP_SF_MMA, false>})
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, kStageSmem);
+        if (e != cudaSuccess) cudaGetLastError();   // no stale error left behind
         attr_err[dev] = e;
     });
     if (attr_err[dev] != cudaSuccess) return BSP_ERR_CUDA;
